@@ -1,0 +1,88 @@
+"""ctypes binding of libkdtopkl.so: the C entry points under the same names.
+
+Argument marshalling only.  Pointers are passed as Python ints (device
+addresses), sizes as ints, the stream as an int (cudaStream_t).  Loading
+fails loudly when the library has not been built: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB
+
+KD_OK = 0
+KD_ERR_INVALID_ARG = 1
+KD_ERR_UNSUPPORTED = 2
+KD_ERR_WORKSPACE = 3
+KD_ERR_CUDA = 4
+KD_ERR_BAD_INDEX = 5
+KD_ERR_TIMEOUT = 6
+
+EXPORTS = (
+    "kd_status_string",
+    "kd_topk_kl_workspace_size",
+    "kd_topk_kl_forward",
+    "kd_topk_kl_backward",
+    "kd_topk_kl_check",
+)
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise ImportError(
+                f"libkdtopkl.so not found at {LIB}; build it with "
+                "`python -m chunked_top_kl_b200.build` (CUDA sm_100a)")
+        lib = ctypes.CDLL(LIB)
+        p, i64, f32, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int, ctypes.c_size_t
+        lib.kd_status_string.argtypes = [i32]
+        lib.kd_status_string.restype = ctypes.c_char_p
+        lib.kd_topk_kl_workspace_size.argtypes = [i64, i64, i64, i64, i64]
+        lib.kd_topk_kl_workspace_size.restype = sz
+        lib.kd_topk_kl_forward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p, sz, p]
+        lib.kd_topk_kl_forward.restype = i32
+        lib.kd_topk_kl_backward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p, p, i32,
+                                            p, sz, p]
+        lib.kd_topk_kl_backward.restype = i32
+        lib.kd_topk_kl_check.argtypes = [p, p, ctypes.POINTER(i64)]
+        lib.kd_topk_kl_check.restype = i32
+        _lib = lib
+    return _lib
+
+
+class KDError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {kd_status_string(status)}")
+
+
+def kd_status_string(status: int) -> str:
+    return load().kd_status_string(int(status)).decode()
+
+
+def kd_topk_kl_workspace_size(N: int, d: int, V: int, K: int, chunk: int) -> int:
+    return int(load().kd_topk_kl_workspace_size(N, d, V, K, chunk))
+
+
+def kd_topk_kl_forward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, loss, lse,
+                       workspace, workspace_bytes, stream) -> int:
+    return int(load().kd_topk_kl_forward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk,
+                                         loss, lse, workspace, workspace_bytes, stream))
+
+
+def kd_topk_kl_backward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse, grad_loss,
+                        dH, dW, accumulate_dW, workspace, workspace_bytes, stream) -> int:
+    return int(load().kd_topk_kl_backward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk,
+                                          lse, grad_loss, dH, dW, int(accumulate_dW), workspace,
+                                          workspace_bytes, stream))
+
+
+def kd_topk_kl_check(workspace, stream) -> tuple[int, int]:
+    n = ctypes.c_int64(0)
+    st = int(load().kd_topk_kl_check(workspace, stream, ctypes.byref(n)))
+    return st, int(n.value)

@@ -1,0 +1,125 @@
+"""Torch-facing wrappers over the C ABI: allocate outputs and workspace with
+torch on the tensors' device, pass raw pointers and the current stream, and
+raise on a non-zero status.  No arithmetic of the loss happens here."""
+
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_inputs(H, W, topk_idx, topk_logit, mask):
+    if not (H.is_cuda and W.is_cuda and topk_idx.is_cuda and topk_logit.is_cuda):
+        raise ValueError("kd_topk_kl: all inputs must be CUDA tensors")
+    if H.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("kd_topk_kl: H and W must be bfloat16")
+    if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
+        raise TypeError("kd_topk_kl: topk_idx must be int32 and topk_logit float32")
+    if mask is not None and (mask.dtype != torch.float32 or not mask.is_cuda):
+        raise TypeError("kd_topk_kl: mask must be a float32 CUDA tensor")
+    for t in (H, W, topk_idx, topk_logit) + ((mask,) if mask is not None else ()):
+        if not t.is_contiguous():
+            raise ValueError("kd_topk_kl: inputs must be contiguous")
+    N, d = H.shape
+    V = W.shape[0]
+    K = topk_idx.shape[1]
+    if W.shape[1] != d or topk_idx.shape != (N, K) or topk_logit.shape != (N, K):
+        raise ValueError("kd_topk_kl: shape mismatch")
+    if mask is not None and mask.shape != (N,):
+        raise ValueError("kd_topk_kl: mask must have shape [N]")
+    return N, d, V, K
+
+
+def workspace_bytes(N: int, d: int, V: int, K: int, chunk: int) -> int:
+    n = _abi.kd_topk_kl_workspace_size(N, d, V, K, chunk)
+    if n == 0:
+        raise ValueError("kd_topk_kl: unsupported sizes")
+    return n
+
+
+def alloc_workspace(N, d, V, K, chunk, device) -> torch.Tensor:
+    return torch.empty(workspace_bytes(N, d, V, K, chunk), dtype=torch.uint8, device=device)
+
+
+def _raise(st: int, where: str):
+    if st != _abi.KD_OK:
+        raise _abi.KDError(st, where)
+
+
+def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
+            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Returns (loss [] fp32, lse [N] fp32)."""
+    N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
+    dev = H.device
+    if workspace is None:
+        workspace = alloc_workspace(N, d, V, K, chunk, dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = _abi.kd_topk_kl_forward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                 N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
+                                 _ptr(workspace), workspace.numel(), stream)
+    _raise(st, "kd_topk_kl_forward")
+    return loss, lse
+
+
+def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.Tensor,
+             grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
+             accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
+             dH: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Returns (dH [N,d] bf16, dW [V,d] fp32)."""
+    N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
+    dev = H.device
+    if workspace is None:
+        workspace = alloc_workspace(N, d, V, K, chunk, dev)
+    if dH is None:
+        dH = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    if dW is None:
+        dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+        accumulate_dW = False
+    if grad_loss is not None:
+        grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                  N, d, V, K, float(T), int(chunk), _ptr(lse), _ptr(grad_loss),
+                                  _ptr(dH), _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
+                                  workspace.numel(), stream)
+    _raise(st, "kd_topk_kl_backward")
+    return dH, dW
+
+
+def check(workspace: torch.Tensor) -> Tuple[int, int]:
+    """Synchronise the current stream and read the device status words:
+    returns (status, bad_index_count)."""
+    stream = torch.cuda.current_stream(workspace.device).cuda_stream
+    return _abi.kd_topk_kl_check(_ptr(workspace), stream)
+
+
+class KDTopKKLFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, H, W, topk_idx, topk_logit, mask, T, chunk):
+        loss, lse = forward(H, W, topk_idx, topk_logit, mask, T, chunk)
+        ctx.save_for_backward(H, W, topk_idx, topk_logit, mask, lse)
+        ctx.T, ctx.chunk = T, chunk
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad):
+        H, W, topk_idx, topk_logit, mask, lse = ctx.saved_tensors
+        dH, dW = backward(H, W, topk_idx, topk_logit, mask, ctx.T, ctx.chunk, lse,
+                          grad_loss=grad.reshape(()))
+        return dH, dW.to(W.dtype), None, None, None, None, None
+
+
+def kd_topk_kl_loss(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096):
+    """Differentiable loss (autograd).  dW is accumulated in fp32 inside the
+    library and cast to W's dtype for autograd; call ``backward`` directly to
+    keep an fp32 gradient."""
+    return KDTopKKLFunction.apply(H, W, topk_idx, topk_logit, mask, T, chunk)

@@ -1,0 +1,473 @@
+// Persistent, warp-specialised tcgen05 GEMM with pluggable epilogues.
+//
+// One CTA per SM.  Warp 0 issues TMA loads into a STAGES-deep shared-memory
+// ring, warp 1 issues tcgen05.mma (bf16 x bf16 -> fp32 in tensor memory),
+// warps 2-5 run the epilogue straight out of tensor memory.  Two 128 x 256
+// fp32 accumulators (all 512 TMEM columns) let the epilogue of one tile
+// overlap the MMAs of the next.
+//
+// Work is a list of units; a unit is one 128-row tile band (m) and a
+// contiguous range of 256-column tiles [n0, n1).  All three roles walk the
+// same unit sequence (u = blockIdx.x, blockIdx.x + gridDim.x, ...), so no
+// scheduling state is shared between them.  The epilogue object lives for a
+// unit, which is what lets the forward epilogue carry a running
+// max / sum-exp across the vocabulary tiles of its range.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kd_ptx.cuh"
+#include "kd_schedule.h"
+#include "kd_small_kernels.cuh"
+
+namespace kd {
+
+constexpr int BM = 128;          // tile rows (TMEM lanes)
+constexpr int BN = 256;          // tile columns (TMEM columns per accumulator)
+constexpr int BK = 64;           // bf16 elements per 128-byte swizzle row
+constexpr int UMMA_K = 16;       // K of one tcgen05.mma kind::f16
+constexpr int STAGES = 4;
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int B_STAGE_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int GEMM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct GemmArgs {
+  Raster raster;
+  int num_kb;           // BK-wide K blocks per tile
+  int a_row0, b_row0;   // tensor-map offsets added to the row (M / N) coordinate
+  int a_k0, b_k0;       // tensor-map offsets added to the K coordinate
+  Status* status;
+};
+
+// Loads one operand tile (rows x BK) for K block kb into shared memory.
+//  K-major: one box {BK, rows} at (k, row).  The smem tile is rows x 128 B,
+//           8-row groups 1024 B apart (SBO), 128-byte swizzled.
+//  MN-major: rows/64 boxes {64, BK} at (row + 64 i, k).  Each box is BK
+//           K-rows of 128 B (64 MN elements); boxes are BK*128 B apart (LBO).
+template <bool MN_MAJOR, int ROWS>
+__device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* tm, int row, int k,
+                                             uint32_t bar) {
+  if constexpr (!MN_MAJOR) {
+    tma_load_2d(dst, tm, k, row, bar);
+  } else {
+#pragma unroll
+    for (int i = 0; i < ROWS / 64; ++i) tma_load_2d(dst + i * (BK * 128), tm, row + 64 * i, k, bar);
+  }
+}
+
+// Descriptor of the kk-th UMMA_K slice of an operand tile in shared memory.
+template <bool MN_MAJOR>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
+  if constexpr (!MN_MAJOR) {
+    // K-major SW128: K advances inside the 128-byte row.
+    return smem_desc_sw128(base + kk * UMMA_K * 2, 16, 1024);
+  } else {
+    // MN-major SW128: K advances by UMMA_K rows of 128 B.
+    return smem_desc_sw128(base + kk * UMMA_K * 128, BK * 128, 1024);
+  }
+}
+
+template <class Epi, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const GemmArgs args, const typename Epi::Params ep) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  const uint32_t bar_base = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar_base + 8u * s; };
+  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Raster& R = args.raster;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4 * 32);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  bool failed = false;
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int u = blockIdx.x; u < R.num_units && !failed; u += gridDim.x) {
+        int m, split, n0, n1;
+        decode_unit(R, u, m, split, n0, n1);
+        for (int n = n0; n < n1 && !failed; ++n) {
+          for (int kb = 0; kb < args.num_kb; ++kb) {
+            if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag)) { failed = true; break; }
+            const uint32_t sa = sbase + stage * STAGE_BYTES;
+            const uint32_t sb = sa + A_STAGE_BYTES;
+            mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+            load_operand<A_MN, BM>(sa, &tmA, args.a_row0 + m * BM, args.a_k0 + kb * BK, full_bar(stage));
+            load_operand<B_MN, BN>(sb, &tmB, args.b_row0 + n * BN, args.b_k0 + kb * BK, full_bar(stage));
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int u = blockIdx.x; u < R.num_units && !failed; u += gridDim.x) {
+        int m, split, n0, n1;
+        decode_unit(R, u, m, split, n0, n1);
+        for (int n = n0; n < n1 && !failed; ++n) {
+          if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { failed = true; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * BN;
+          for (int kb = 0; kb < args.num_kb; ++kb) {
+            if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag)) { failed = true; break; }
+            tc_fence_after();
+            const uint32_t sa = sbase + stage * STAGE_BYTES;
+            const uint32_t sb = sa + A_STAGE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+              tc_mma_bf16(d_tmem, operand_desc<A_MN>(sa, kk), operand_desc<B_MN>(sb, kk), idesc,
+                          (kb | kk) != 0 ? 1u : 0u);
+            }
+            tc_commit(empty_bar(stage));
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+          if (failed) break;
+          tc_commit(tfull_bar(acc));
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;          // tile row owned by this thread
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    Epi epi;
+    for (int u = blockIdx.x; u < R.num_units && !failed; u += gridDim.x) {
+      int m, split, n0, n1;
+      decode_unit(R, u, m, split, n0, n1);
+      epi.begin_unit(ep, m, split, n0, row);
+      for (int n = n0; n < n1; ++n) {
+        // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes.
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag));
+        if (!ok) { failed = true; break; }
+        tc_fence_after();
+        epi.tile(ep, m, n, row, lane_addr + acc * BN);
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (failed) break;
+      epi.end_unit(ep, m, split, row);
+    }
+  }
+
+  if (failed) {
+    *abort_flag = 1;
+    atomicOr(&args.status->timeout, 1u);
+  }
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag) {
+    // Let asynchronous copies and MMAs that were already issued land before
+    // the CTA releases its shared and tensor memory.
+    if (warp == 1 && lane == 0) {
+      const uint32_t drain = tfull_bar(0);
+      tc_commit(drain);
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) { }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- epilogues
+
+__device__ __forceinline__ int lower_bound_row(const int32_t* row, int len, int key) {
+  int lo = 0, hi = len;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (row[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// Forward: running max / sum-exp over the unit's vocabulary columns and the
+// gathered sum of p * z at the teacher's columns; one (m, s, g) partial per
+// token per split.  Columns >= V are -inf.
+struct EpiFwd {
+  struct Params {
+    int N, V, Kp;
+    const int32_t* tidx;
+    const float* tp;
+    float* part_m;
+    float* part_s;
+    float* part_g;
+  };
+  float mrun, srun, grun, np;
+  int cur, nidx, grow;
+  const int32_t* trow;
+  const float* prow;
+
+  __device__ __forceinline__ void begin_unit(const Params& P, int m, int, int n0, int row) {
+    grow = m * BM + row;
+    mrun = -INFINITY;
+    srun = 0.f;
+    grun = 0.f;
+    nidx = kSentinel;
+    np = 0.f;
+    if (grow < P.N) {
+      trow = P.tidx + (size_t)grow * P.Kp;
+      prow = P.tp + (size_t)grow * P.Kp;
+      cur = lower_bound_row(trow, P.Kp, n0 * BN);
+      nidx = trow[cur];
+      np = prow[cur];
+    }
+  }
+
+  __device__ __forceinline__ void tile(const Params& P, int, int n, int, uint32_t taddr) {
+#pragma unroll 1
+    for (int j = 0; j < BN / 32; ++j) {
+      float v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + j * 32, v);
+      const int c0 = n * BN + j * 32;
+      if (c0 + 32 > P.V) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c0 + i >= P.V) v[i] = -INFINITY;
+      }
+      if (nidx < c0 + 32) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (c0 + i == nidx) {
+            grun += np * v[i];
+            ++cur;
+            nidx = trow[cur];
+            np = prow[cur];
+          }
+        }
+      }
+      float cm = v[0];
+#pragma unroll
+      for (int i = 1; i < 32; ++i) cm = fmaxf(cm, v[i]);
+      const float mn = fmaxf(mrun, cm);
+      if (mn == -INFINITY) continue;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc += __expf(v[i] - mn);
+      srun = srun * __expf(mrun - mn) + acc;
+      mrun = mn;
+    }
+  }
+
+  __device__ __forceinline__ void end_unit(const Params& P, int, int split, int) {
+    if (grow < P.N) {
+      const size_t o = (size_t)split * P.N + grow;
+      P.part_m[o] = mrun;
+      P.part_s[o] = srun;
+      P.part_g[o] = grun;
+    }
+  }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Backward, per chunk: dZ = c_n (exp(z - lse_n) - p at the teacher's columns),
+// rounded to bf16 and stored for the chunk's tokens (row-major, ldz columns;
+// columns in [V, ldz) are written as 0).
+struct EpiDz {
+  struct Params {
+    int rows_valid;        // tokens in this chunk
+    int row0;              // global token index of chunk row 0
+    int V, ldz, Kp;
+    const int32_t* tidx;
+    const float* tp;
+    const float* lse;
+    const float* mask;     // may be null
+    const float* cscale;   // device scalar g / sum(mask)
+    __nv_bfloat16* dz;
+  };
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, int) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int, int) {}
+
+  __device__ __forceinline__ void tile(const Params& P, int m, int n, int row, uint32_t taddr) {
+    const int r = m * BM + row;
+    const bool valid = r < P.rows_valid;
+    const int grow = P.row0 + r;
+    float L = 0.f, c = 0.f;
+    const int32_t* trow = nullptr;
+    const float* prow = nullptr;
+    int cur = 0, nidx = kSentinel;
+    float np = 0.f;
+    if (valid) {
+      L = P.lse[grow];
+      c = (P.mask ? P.mask[grow] : 1.f) * (*P.cscale);
+      trow = P.tidx + (size_t)grow * P.Kp;
+      prow = P.tp + (size_t)grow * P.Kp;
+      cur = lower_bound_row(trow, P.Kp, n * BN);
+      nidx = trow[cur];
+      np = prow[cur];
+    }
+    __nv_bfloat16* out = P.dz + (size_t)r * P.ldz;
+#pragma unroll 1
+    for (int j = 0; j < BN / 32; ++j) {
+      float v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + j * 32, v);
+      const int c0 = n * BN + j * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __expf(v[i] - L);
+      if (nidx < c0 + 32) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (c0 + i == nidx) {
+            v[i] -= np;
+            ++cur;
+            nidx = trow[cur];
+            np = prow[cur];
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = (c0 + i < P.V) ? c * v[i] : 0.f;
+      if (valid) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (c0 + 8 * t + 8 <= P.ldz) {
+            uint4 w;
+            w.x = pack_bf16x2(v[8 * t + 0], v[8 * t + 1]);
+            w.y = pack_bf16x2(v[8 * t + 2], v[8 * t + 3]);
+            w.z = pack_bf16x2(v[8 * t + 4], v[8 * t + 5]);
+            w.w = pack_bf16x2(v[8 * t + 6], v[8 * t + 7]);
+            *reinterpret_cast<uint4*>(out + c0 + 8 * t) = w;
+          }
+        }
+      }
+    }
+  }
+};
+
+// Backward, per chunk: dH rows of the chunk's tokens, bf16.
+struct EpiDh {
+  struct Params {
+    int rows_valid, row0, d;
+    __nv_bfloat16* dH;
+  };
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, int) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int, int) {}
+
+  __device__ __forceinline__ void tile(const Params& P, int m, int n, int row, uint32_t taddr) {
+    const int r = m * BM + row;
+    const bool valid = r < P.rows_valid;
+    __nv_bfloat16* out = P.dH + (size_t)(P.row0 + r) * P.d;
+#pragma unroll 1
+    for (int j = 0; j < BN / 32; ++j) {
+      float v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + j * 32, v);
+      const int c0 = n * BN + j * 32;
+      if (valid) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (c0 + 8 * t + 8 <= P.d) {
+            uint4 w;
+            w.x = pack_bf16x2(v[8 * t + 0], v[8 * t + 1]);
+            w.y = pack_bf16x2(v[8 * t + 2], v[8 * t + 3]);
+            w.z = pack_bf16x2(v[8 * t + 4], v[8 * t + 5]);
+            w.w = pack_bf16x2(v[8 * t + 6], v[8 * t + 7]);
+            *reinterpret_cast<uint4*>(out + c0 + 8 * t) = w;
+          }
+        }
+      }
+    }
+  }
+};
+
+// Backward, per chunk: dW (+)= dZ^T H for 128 vocabulary rows x 256 columns.
+struct EpiDw {
+  struct Params {
+    int rows_valid, d, accumulate;
+    float* dW;
+  };
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, int) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int, int) {}
+
+  __device__ __forceinline__ void tile(const Params& P, int m, int n, int row, uint32_t taddr) {
+    const int r = m * BM + row;
+    const bool valid = r < P.rows_valid;
+    float* out = P.dW + (size_t)r * P.d;
+#pragma unroll 1
+    for (int j = 0; j < BN / 32; ++j) {
+      float v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + j * 32, v);
+      const int c0 = n * BN + j * 32;
+      if (valid) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (c0 + 4 * t + 4 <= P.d) {
+            float4* p = reinterpret_cast<float4*>(out + c0 + 4 * t);
+            float4 w = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+            if (P.accumulate) {
+              const float4 o = *p;
+              w.x += o.x; w.y += o.y; w.z += o.z; w.w += o.w;
+            }
+            *p = w;
+          }
+        }
+      }
+    }
+  }
+};
+
+}  // namespace kd

@@ -1,0 +1,349 @@
+// Host side of libkdtopkl.so: argument checks, workspace layout, TMA tensor
+// maps, schedules and kernel launches for the fused chunked top-K KL loss.
+//
+// Forward (one call):  teacher_prep -> gemm<EpiFwd> -> lse_merge -> finalize
+// Backward (one call): teacher_prep -> finalize(scale) -> for each chunk of
+//                      tokens: gemm<EpiDz> -> gemm<EpiDh> -> gemm<EpiDw>
+// The fused chunked loss of "Efficient Knowledge Distillation for LLMs"
+// (Japanese summary, method paragraph) projects, normalises and gathers one
+// chunk at a time and recomputes each chunk in the backward pass; here the
+// forward never stores logits at all (the vocabulary tiles live only in
+// tensor memory) and the backward stores one chunk of bf16 dZ.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/kd_topk_kl.h"
+#include "kd_gemm.cuh"
+#include "kd_small_kernels.cuh"
+
+using namespace kd;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+struct Layout {
+  int Kp = 0;
+  int64_t ldz = 0, C = 0;
+  int64_t n_prep_blocks = 0, n_merge_blocks = 0;
+  size_t off_status = 0, off_scal = 0, off_mask_part = 0, off_term_part = 0;
+  size_t off_tidx = 0, off_tp = 0, off_ent = 0, off_pm = 0, off_ps = 0, off_pg = 0, off_dz = 0;
+  size_t total = 0;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout make_layout(int64_t N, int64_t V, int64_t K, int64_t chunk) {
+  Layout L;
+  L.Kp = (int)round_up(K + 1, 4);
+  L.ldz = round_up(V, 8);
+  L.C = N > 0 ? (chunk < N ? chunk : N) : 1;
+  L.n_prep_blocks = ceil_div(N > 0 ? N : 1, kPrepWarps);
+  L.n_merge_blocks = ceil_div(N > 0 ? N : 1, kMergeThreads);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
+  L.off_status = take(sizeof(Status));
+  L.off_scal = take(64);
+  L.off_mask_part = take(sizeof(double) * L.n_prep_blocks);
+  L.off_term_part = take(sizeof(double) * L.n_merge_blocks);
+  L.off_tidx = take(sizeof(int32_t) * (size_t)N * L.Kp);
+  L.off_tp = take(sizeof(float) * (size_t)N * L.Kp);
+  L.off_ent = take(sizeof(float) * (size_t)N);
+  L.off_pm = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_dz = take(2 * (size_t)L.C * L.ldz);
+  L.total = o;
+  return L;
+}
+
+int check_shapes(int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk) {
+  if (N < 0 || d <= 0 || V <= 0 || K <= 0 || chunk <= 0) return KD_ERR_INVALID_ARG;
+  if (!(T > 0.f) || !(T < INFINITY)) return KD_ERR_INVALID_ARG;
+  if (d % 8 != 0 || d < 8) return KD_ERR_UNSUPPORTED;
+  if (K > kMaxK) return KD_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || d >= (int64_t(1) << 24))
+    return KD_ERR_UNSUPPORTED;
+  return KD_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------- TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [outer][inner] with row pitch `pitch` elements,
+// 128-byte-swizzled boxes of box_inner x box_outer, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+              uint32_t box_inner, uint32_t box_outer) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- device info
+
+struct DevInfo {
+  int sms = 0;
+  bool attr_set[8] = {};
+};
+DevInfo g_dev[kMaxDevices];
+
+int device_sms(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_dev[dev].sms) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    g_dev[dev].sms = v > 0 ? v : 148;
+  }
+  return g_dev[dev].sms;
+}
+
+template <class Epi, bool A_MN, bool B_MN>
+cudaError_t launch_gemm(int slot, int dev, int grid, const CUtensorMap& ta, const CUtensorMap& tb,
+                        const GemmArgs& args, const typename Epi::Params& ep, cudaStream_t s) {
+  auto kern = gemm_tc_kernel<Epi, A_MN, B_MN>;
+  if (dev >= 0 && dev < kMaxDevices && !g_dev[dev].attr_set[slot]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    g_dev[dev].attr_set[slot] = true;
+  }
+  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, args, ep);
+  return cudaGetLastError();
+}
+
+inline int grid_for(const Raster& r, int sms) { return r.num_units < sms ? r.num_units : sms; }
+
+int common_checks(const void* H, const void* W, const int32_t* idx, const float* logit,
+                  int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                  void* ws, size_t ws_bytes, Layout* L) {
+  int st = check_shapes(N, d, V, K, T, chunk);
+  if (st != KD_OK) return st;
+  if (!W || !ws) return KD_ERR_INVALID_ARG;
+  if (N > 0 && (!H || !idx || !logit)) return KD_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || (H && !aligned(H, 16)) || !aligned(ws, 256)) return KD_ERR_INVALID_ARG;
+  if ((idx && !aligned(idx, 4)) || (logit && !aligned(logit, 4))) return KD_ERR_INVALID_ARG;
+  *L = make_layout(N, V, K, chunk);
+  if (ws_bytes < L->total) return KD_ERR_WORKSPACE;
+  return KD_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+}  // namespace
+
+extern "C" {
+
+const char* kd_status_string(int s) {
+  switch (s) {
+    case KD_OK: return "KD_OK";
+    case KD_ERR_INVALID_ARG: return "KD_ERR_INVALID_ARG";
+    case KD_ERR_UNSUPPORTED: return "KD_ERR_UNSUPPORTED";
+    case KD_ERR_WORKSPACE: return "KD_ERR_WORKSPACE";
+    case KD_ERR_CUDA: return "KD_ERR_CUDA";
+    case KD_ERR_BAD_INDEX: return "KD_ERR_BAD_INDEX";
+    case KD_ERR_TIMEOUT: return "KD_ERR_TIMEOUT";
+    default: return "KD_ERR_UNKNOWN";
+  }
+}
+
+size_t kd_topk_kl_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
+  if (check_shapes(N, d, V, K, 1.0f, chunk) != KD_OK) return 0;
+  return make_layout(N, V, K, chunk).total;
+}
+
+int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
+                       const float* topk_logit, const float* mask, int64_t N, int64_t d,
+                       int64_t V, int64_t K, float T, int64_t chunk, float* loss, float* lse,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  Layout L;
+  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
+                         workspace_bytes, &L);
+  if (st != KD_OK) return st;
+  if (!loss || (N > 0 && !lse)) return KD_ERR_INVALID_ARG;
+  if (mask && !aligned(mask, 4)) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
+
+  if (cudaMemsetAsync(at<Status>(workspace, L.off_status), 0, sizeof(Status), s) != cudaSuccess)
+    return KD_ERR_CUDA;
+  if (N == 0) {
+    return cudaMemsetAsync(loss, 0, sizeof(float), s) == cudaSuccess ? KD_OK : KD_ERR_CUDA;
+  }
+  Status* status = at<Status>(workspace, L.off_status);
+  int32_t* tidx = at<int32_t>(workspace, L.off_tidx);
+  float* tp = at<float>(workspace, L.off_tp);
+  float* ent = at<float>(workspace, L.off_ent);
+  double* mask_part = at<double>(workspace, L.off_mask_part);
+  double* term_part = at<double>(workspace, L.off_term_part);
+
+  teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
+      topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+  if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+
+  CUtensorMap tmH, tmW;
+  if (!make_map(&tmH, H, d, N, d, BK, BM) || !make_map(&tmW, W, d, V, d, BK, BN))
+    return KD_ERR_CUDA;
+  const int sms = device_sms(dev);
+  GemmArgs a{};
+  a.raster = forward_raster(ceil_div(N, BM), ceil_div(V, BN), sms);
+  a.num_kb = (int)ceil_div(d, BK);
+  a.status = status;
+  EpiFwd::Params ep{};
+  ep.N = (int)N;
+  ep.V = (int)V;
+  ep.Kp = L.Kp;
+  ep.tidx = tidx;
+  ep.tp = tp;
+  ep.part_m = at<float>(workspace, L.off_pm);
+  ep.part_s = at<float>(workspace, L.off_ps);
+  ep.part_g = at<float>(workspace, L.off_pg);
+  if (launch_gemm<EpiFwd, false, false>(0, dev, grid_for(a.raster, sms), tmH, tmW, a, ep, s) != cudaSuccess)
+    return KD_ERR_CUDA;
+
+  lse_merge_kernel<<<(unsigned)L.n_merge_blocks, kMergeThreads, 0, s>>>(
+      ep.part_m, ep.part_s, ep.part_g, a.raster.splits, (int)N, ent, mask, lse, term_part);
+  finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, term_part,
+                                    (int)L.n_merge_blocks, 0, nullptr, loss);
+  return cudaGetLastError() == cudaSuccess ? KD_OK : KD_ERR_CUDA;
+}
+
+int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
+                        const float* topk_logit, const float* mask, int64_t N, int64_t d,
+                        int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
+                        const float* grad_loss, void* dH, float* dW, int accumulate_dW,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  Layout L;
+  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
+                         workspace_bytes, &L);
+  if (st != KD_OK) return st;
+  if (!dW || !aligned(dW, 16)) return KD_ERR_INVALID_ARG;
+  if (N > 0 && (!lse || !dH || !aligned(dH, 16))) return KD_ERR_INVALID_ARG;
+  if ((mask && !aligned(mask, 4)) || (grad_loss && !aligned(grad_loss, 4))) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
+
+  if (cudaMemsetAsync(at<Status>(workspace, L.off_status), 0, sizeof(Status), s) != cudaSuccess)
+    return KD_ERR_CUDA;
+  if (N == 0) {
+    if (!accumulate_dW && cudaMemsetAsync(dW, 0, sizeof(float) * (size_t)V * d, s) != cudaSuccess)
+      return KD_ERR_CUDA;
+    return KD_OK;
+  }
+  Status* status = at<Status>(workspace, L.off_status);
+  int32_t* tidx = at<int32_t>(workspace, L.off_tidx);
+  float* tp = at<float>(workspace, L.off_tp);
+  float* ent = at<float>(workspace, L.off_ent);
+  double* mask_part = at<double>(workspace, L.off_mask_part);
+  float* cscale = at<float>(workspace, L.off_scal);
+  __nv_bfloat16* dz = at<__nv_bfloat16>(workspace, L.off_dz);
+
+  teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
+      topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+  finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, nullptr, 0, 1, grad_loss, cscale);
+  if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+
+  CUtensorMap tmHk, tmWk, tmWmn, tmHmn;
+  if (!make_map(&tmHk, H, d, N, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, BN) ||
+      !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, H, d, N, d, 64, BK))
+    return KD_ERR_CUDA;
+  const int sms = device_sms(dev);
+
+  for (int64_t c0 = 0; c0 < N; c0 += chunk) {
+    const int64_t Cc = (N - c0 < chunk) ? (N - c0) : chunk;
+    CUtensorMap tmZk, tmZmn;
+    if (!make_map(&tmZk, dz, L.ldz, Cc, L.ldz, BK, BM) || !make_map(&tmZmn, dz, L.ldz, Cc, L.ldz, 64, BK))
+      return KD_ERR_CUDA;
+
+    // dZ for the chunk: recompute z = H W^T tile by tile.
+    GemmArgs a3{};
+    a3.raster = tile_raster(ceil_div(Cc, BM), ceil_div(V, BN), true);
+    a3.num_kb = (int)ceil_div(d, BK);
+    a3.a_row0 = (int)c0;
+    a3.status = status;
+    EpiDz::Params e3{};
+    e3.rows_valid = (int)Cc;
+    e3.row0 = (int)c0;
+    e3.V = (int)V;
+    e3.ldz = (int)L.ldz;
+    e3.Kp = L.Kp;
+    e3.tidx = tidx;
+    e3.tp = tp;
+    e3.lse = lse;
+    e3.mask = mask;
+    e3.cscale = cscale;
+    e3.dz = dz;
+    if (launch_gemm<EpiDz, false, false>(1, dev, grid_for(a3.raster, sms), tmHk, tmWk, a3, e3, s) != cudaSuccess)
+      return KD_ERR_CUDA;
+
+    // dH[chunk] = dZ W   (A = dZ, K-major over V; B = W, MN-major over d).
+    GemmArgs a4{};
+    a4.raster = tile_raster(ceil_div(Cc, BM), ceil_div(d, BN), true);
+    a4.num_kb = (int)ceil_div(V, BK);
+    a4.status = status;
+    EpiDh::Params e4{};
+    e4.rows_valid = (int)Cc;
+    e4.row0 = (int)c0;
+    e4.d = (int)d;
+    e4.dH = static_cast<__nv_bfloat16*>(dH);
+    if (launch_gemm<EpiDh, false, true>(2, dev, grid_for(a4.raster, sms), tmZk, tmWmn, a4, e4, s) != cudaSuccess)
+      return KD_ERR_CUDA;
+
+    // dW (+)= dZ^T H[chunk]   (A = dZ^T, MN-major over V; B = H, MN-major over d).
+    GemmArgs a5{};
+    a5.raster = tile_raster(ceil_div(V, BM), ceil_div(d, BN), false);
+    a5.num_kb = (int)ceil_div(Cc, BK);
+    a5.b_k0 = (int)c0;
+    a5.status = status;
+    EpiDw::Params e5{};
+    e5.rows_valid = (int)V;
+    e5.d = (int)d;
+    e5.accumulate = (accumulate_dW || c0 > 0) ? 1 : 0;
+    e5.dW = dW;
+    if (launch_gemm<EpiDw, true, true>(3, dev, grid_for(a5.raster, sms), tmZmn, tmHmn, a5, e5, s) != cudaSuccess)
+      return KD_ERR_CUDA;
+  }
+  return KD_OK;
+}
+
+int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_count) {
+  if (!workspace) return KD_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KD_ERR_CUDA;
+  Status h;
+  if (cudaMemcpy(&h, workspace, sizeof(Status), cudaMemcpyDeviceToHost) != cudaSuccess) return KD_ERR_CUDA;
+  if (bad_index_count) *bad_index_count = (int64_t)h.bad_index;
+  if (h.timeout) return KD_ERR_TIMEOUT;
+  if (h.bad_index) return KD_ERR_BAD_INDEX;
+  return KD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,121 @@
+/*
+ * kd_topk_kl.h - C ABI of the fused chunked top-K KL distillation loss
+ * (libkdtopkl.so, CUDA sm_100a).
+ *
+ * The operation is the one of "Efficient Knowledge Distillation for LLMs:
+ * Offline Top-K Logits and a Fused Chunked KL Loss": the student is trained
+ * against an offline cache of the teacher's top-K logits per position
+ * (blog post, "Two systems changes", offline distillation paragraph) with a
+ * KL loss whose output projection is fused into the loss and recomputed per
+ * chunk in the backward pass, so that the N x V logit grid is never stored
+ * and peak memory is linear in the number of tokens (Japanese summary,
+ * method paragraph: the fused chunked variant; abstract).
+ *
+ * For student hidden states H[N,d], LM-head weight W[V,d], teacher cache
+ * (idx[N,K], logit[N,K]), mask m[N], temperature T:
+ *   z[n,v]  = sum_j H[n,j] W[v,j]
+ *   lse[n]  = log sum_v exp(z[n,v])
+ *   p[n,k]  = softmax_k(logit[n,k] / T)
+ *   term[n] = sum_k p[n,k] (log p[n,k] - (z[n,idx[n,k]] - lse[n]))
+ *   loss    = sum_n m[n] term[n] / sum_n m[n]        (0 when sum m = 0)
+ * and, for an upstream scalar g,
+ *   dZ[n,v] = g m[n] / sum m * (exp(z[n,v] - lse[n]) - sum_{k: idx[n,k]=v} p[n,k])
+ *   dH      = dZ W            dW (+)= dZ^T H
+ * T divides the teacher logits only.  Duplicate teacher indices add their
+ * probabilities at that column (the loss keeps the per-slot sum).
+ *
+ * Conventions shared by every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller.  The
+ *    library never allocates device or host memory and keeps no state
+ *    between calls except a per-device, per-kernel attribute cache.
+ *  - Layouts are dense row-major: H bf16 [N][d], W bf16 [V][d],
+ *    topk_idx int32 [N][K], topk_logit fp32 [N][K], mask fp32 [N],
+ *    lse fp32 [N], dH bf16 [N][d], dW fp32 [V][d].  bf16 is IEEE bfloat16
+ *    stored as uint16.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls
+ *    enqueue work and return without synchronising.  Argument errors are
+ *    reported synchronously by the return value and nothing is enqueued.
+ *  - Supported shapes: N >= 0, 1 <= V < 2^31, d >= 8 with d % 8 == 0,
+ *    1 <= K <= 512, T > 0 and finite, chunk >= 1.  H, W, dH and dW must be
+ *    16-byte aligned, the workspace 256-byte aligned.
+ *  - Teacher indices outside [0, V) are not an argument error: they are
+ *    dropped (contribute nothing), counted in the workspace and reported by
+ *    kd_topk_kl_check as KD_ERR_BAD_INDEX; the results are then undefined
+ *    in value but every memory access stays in bounds.
+ *  - Results are deterministic: the same inputs give bitwise the same
+ *    outputs on every run (fixed-order reductions, no float atomics).
+ *  - A workspace may be used by one call at a time (calls on one stream
+ *    are serialised; calls on different streams need different workspaces).
+ */
+#ifndef KD_TOPK_KL_H
+#define KD_TOPK_KL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kd_status {
+  KD_OK = 0,
+  KD_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad alignment, T <= 0 */
+  KD_ERR_UNSUPPORTED = 2,  /* shape outside the supported set (d % 8, K > 512, ...) */
+  KD_ERR_WORKSPACE = 3,    /* workspace_bytes smaller than kd_topk_kl_workspace_size */
+  KD_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  KD_ERR_BAD_INDEX = 5,    /* (from kd_topk_kl_check) a teacher index was outside [0, V) */
+  KD_ERR_TIMEOUT = 6       /* (from kd_topk_kl_check) a pipeline wait gave up; results invalid */
+} kd_status;
+
+/* Human-readable name of a status code.  Never returns NULL. */
+const char* kd_status_string(int status);
+
+/* Bytes of device workspace that kd_topk_kl_forward / kd_topk_kl_backward
+ * need for these sizes (the same workspace size serves both).  Returns 0
+ * for sizes that the entry points would reject.  It holds the prepared
+ * teacher cache (sorted indices and probabilities, N x (K+1..K+4) x 8 B),
+ * per-token partial log-sum-exp state, and one chunk of dZ
+ * (chunk x round_up(V, 8) bf16): linear in N, and in chunk x V. */
+size_t kd_topk_kl_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk);
+
+/* Forward pass.  Writes *loss (device fp32 scalar) and lse[N] (device fp32;
+ * every token's student log-sum-exp, masked tokens included), which the
+ * backward pass consumes.  mask may be NULL (all ones).  The logit grid is
+ * never stored: each vocabulary tile of z = H W^T lives only in tensor
+ * memory while its running max / sum-exp and the teacher gather are updated
+ * (Japanese summary, method paragraph: fused chunked KL). */
+int kd_topk_kl_forward(const void* H, const void* W,
+                       const int32_t* topk_idx, const float* topk_logit,
+                       const float* mask,
+                       int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                       float* loss, float* lse,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward pass.  Recomputes z chunk by chunk (chunk tokens at a time; the
+ * pages' "recompute each chunk during the backward pass", Japanese
+ * summary, method paragraph), forms dZ for that chunk only, and writes
+ * dH (bf16 [N][d], overwritten) and dW (fp32 [V][d]; overwritten when
+ * accumulate_dW == 0, added to when accumulate_dW != 0).  lse must be the
+ * forward pass's output for the same inputs.  grad_loss is a device fp32
+ * scalar (the upstream gradient of the loss) or NULL for 1.0.  dZ is
+ * rounded to bf16 before the two gradient products. */
+int kd_topk_kl_backward(const void* H, const void* W,
+                        const int32_t* topk_idx, const float* topk_logit,
+                        const float* mask,
+                        int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                        const float* lse, const float* grad_loss,
+                        void* dH, float* dW, int accumulate_dW,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the device-side status words that the
+ * last forward or backward call on this workspace wrote.  Returns KD_OK,
+ * KD_ERR_BAD_INDEX (teacher index outside [0, V) seen), KD_ERR_TIMEOUT (a
+ * bounded pipeline wait expired), or KD_ERR_CUDA.  If bad_index_count is
+ * not NULL it receives the number of out-of-range teacher indices. */
+int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KD_TOPK_KL_H */

@@ -1,0 +1,55 @@
+// Enumerates the GEMM tile schedules of kd_schedule.h for a list of shapes
+// and checks that every output tile is visited exactly once, that every
+// unit has a non-empty column range, and that the forward schedule keeps
+// within its split limit.  Prints "OK <cases>" or the first failure.
+#include <cstdio>
+#include <vector>
+
+#include "../../chunked_top_kl_b200/csrc/kd_schedule.h"
+
+using namespace kd;
+
+static bool check(const Raster& r, const char* what, long a, long b, long c) {
+  if (r.num_units != r.m_tiles * r.splits) { printf("FAIL %s units %ld %ld %ld\n", what, a, b, c); return false; }
+  std::vector<int> seen((size_t)r.m_tiles * r.n_tiles, 0);
+  for (int u = 0; u < r.num_units; ++u) {
+    int m, s, n0, n1;
+    decode_unit(r, u, m, s, n0, n1);
+    if (m < 0 || m >= r.m_tiles || s < 0 || s >= r.splits || n0 < 0 || n0 >= n1 || n1 > r.n_tiles) {
+      printf("FAIL %s unit %d -> m %d s %d [%d,%d) for %ld %ld %ld\n", what, u, m, s, n0, n1, a, b, c);
+      return false;
+    }
+    for (int n = n0; n < n1; ++n) seen[(size_t)m * r.n_tiles + n]++;
+  }
+  for (size_t i = 0; i < seen.size(); ++i)
+    if (seen[i] != 1) { printf("FAIL %s tile %zu seen %d for %ld %ld %ld\n", what, i, seen[i], a, b, c); return false; }
+  return true;
+}
+
+int main() {
+  const long Ns[] = {1, 127, 128, 129, 512, 1000, 4096, 8192, 32768, 65536, 262144};
+  const long Vs[] = {1, 24, 255, 256, 257, 4096, 32000, 128256, 201088};
+  const long ds[] = {8, 72, 256, 2048, 2880, 3072};
+  const long chunks[] = {1, 64, 128, 1000, 1024, 2048, 4096};
+  const int grids[] = {1, 7, 148};
+  int cases = 0;
+  for (long N : Ns)
+    for (long V : Vs)
+      for (int g : grids) {
+        Raster r = forward_raster(ceil_div64(N, 128), ceil_div64(V, 256), g);
+        if (r.splits > kMaxSplits) { printf("FAIL splits %d\n", r.splits); return 1; }
+        if (r.group_m < 1) { printf("FAIL group_m\n"); return 1; }
+        if (!check(r, "fwd", N, V, g)) return 1;
+        ++cases;
+      }
+  for (long C : chunks)
+    for (long V : Vs)
+      for (long d : ds) {
+        if (!check(tile_raster(ceil_div64(C, 128), ceil_div64(V, 256), true), "dz", C, V, d)) return 1;
+        if (!check(tile_raster(ceil_div64(C, 128), ceil_div64(d, 256), true), "dh", C, V, d)) return 1;
+        if (!check(tile_raster(ceil_div64(V, 128), ceil_div64(d, 256), false), "dw", C, V, d)) return 1;
+        cases += 3;
+      }
+  printf("OK %d\n", cases);
+  return 0;
+}

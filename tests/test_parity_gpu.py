@@ -1,0 +1,218 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element.
+
+Tolerances: loss relative error <= 1e-3, per-token lse absolute error
+<= 2e-3, relative Frobenius error <= 1e-2 for dH and dW.  Small and ragged
+shapes are compared in full; the large workloads on sampled rows (the oracle
+computes those one by one) and on identities that hold at any size.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from workloads.configs import Config
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-3
+LSE_ATOL = 2e-3
+GRAD_RFRO = 1e-2
+
+
+@pytest.fixture(scope="module")
+def kd():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from chunked_top_kl_b200 import build
+    build.build()
+    import chunked_top_kl_b200 as k
+    return k
+
+
+def _cfg(N, d, V, K, T=1.0, chunk=128, seed=0, mask="ones", teacher="uniform", w_std=None):
+    return Config(f"case_N{N}_d{d}_V{V}_K{K}", N, d, V, K, T, chunk,
+                  w_std=(w_std if w_std is not None else d ** -0.5), teacher=teacher, mask=mask, seed=seed)
+
+
+def _to_dev(x):
+    return {k: v.cuda() for k, v in x.items()}
+
+
+def _gpu(kd, x, T, chunk, grad=None, mask=True):
+    g = _to_dev(x)
+    m = g["mask"] if mask else None
+    ws = kd.alloc_workspace(g["H"].shape[0], g["H"].shape[1], g["W"].shape[0], g["topk_idx"].shape[1],
+                            chunk, g["H"].device)
+    loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], m, T, chunk, workspace=ws)
+    st, nbad = kd.check(ws)
+    assert st == 0, kd.kd_status_string(st)
+    gl = None if grad is None else torch.tensor(grad, dtype=torch.float32, device="cuda")
+    dH, dW = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], m, T, chunk, lse,
+                         grad_loss=gl, workspace=ws)
+    st, nbad = kd.check(ws)
+    assert st == 0, kd.kd_status_string(st)
+    torch.cuda.synchronize()
+    return {"loss": float(loss.item()), "lse": lse.cpu().double().numpy(),
+            "dH": dH.float().cpu().double().numpy(), "dW": dW.cpu().double().numpy()}
+
+
+def _rfro(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def _assert_parity(got, ref, what=""):
+    rel = abs(got["loss"] - ref["loss"]) / max(abs(ref["loss"]), 1e-30)
+    assert rel <= LOSS_RTOL, f"{what} loss {got['loss']} vs {ref['loss']} (rel {rel:.2e})"
+    lse_err = np.max(np.abs(got["lse"] - ref["lse"]))
+    assert lse_err <= LSE_ATOL, f"{what} lse max abs err {lse_err:.2e}"
+    for k in ("dH", "dW"):
+        e = _rfro(got[k], ref[k])
+        assert e <= GRAD_RFRO, f"{what} {k} rel Frobenius err {e:.2e}"
+
+
+def _oracle(x, T, grad=1.0, mask=True):
+    return oracle.kd_topk_kl(x["H"], x["W"], x["topk_idx"], x["topk_logit"],
+                             x["mask"] if mask else None, T, grad=grad)
+
+
+SMALL_CASES = [
+    # (N, d, V, K, T, chunk, mask)   ragged in every dimension somewhere
+    (512, 256, 4096, 16, 1.0, 128, "ones"),          # the small parity workload's shape
+    (300, 72, 1000, 7, 0.7, 100, "drop5"),            # ragged N, d, V; 3 chunks + tail
+    (129, 128, 257, 1, 1.0, 64, "ones"),              # K = 1, one column past a tile
+    (1, 64, 24, 5, 2.0, 4096, "ones"),                # single token, V < one tile
+    (700, 512, 5000, 100, 1.3, 256, "drop5"),         # K = 100, many tiles
+    (256, 8, 300, 300, 1.0, 128, "ones"),             # K = V (whole vocabulary), d = 8
+]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: "N{}_d{}_V{}_K{}".format(*c[:4]))
+def test_parity_small(kd, case):
+    N, d, V, K, T, chunk, mask = case
+    x = workloads.make_inputs(_cfg(N, d, V, K, T=T, chunk=chunk, mask=mask, seed=N + V))
+    ref = _oracle(x, T, grad=1.0)
+    got = _gpu(kd, x, T, chunk)
+    _assert_parity(got, ref, str(case))
+
+
+def test_parity_config0_with_grad_and_no_mask(kd):
+    cfg = workloads.get_config(0)
+    x = workloads.make_inputs(cfg)
+    ref = _oracle(x, cfg.T, grad=2.5, mask=False)
+    got = _gpu(kd, x, cfg.T, cfg.chunk, grad=2.5, mask=False)
+    _assert_parity(got, ref, "config0 grad=2.5")
+
+
+def test_parity_packed_head_config1(kd):
+    cfg = workloads.get_config(1)
+    x = workloads.make_inputs(cfg)
+    ref = _oracle(x, cfg.T)
+    got = _gpu(kd, x, cfg.T, cfg.chunk)
+    _assert_parity(got, ref, "config1")
+    # masked tokens have exactly zero gradient rows
+    masked = (x["mask"].numpy() == 0)
+    assert np.all(got["dH"][masked] == 0.0)
+
+
+def test_chunk_invariance_and_determinism(kd):
+    x = workloads.make_inputs(_cfg(300, 72, 1000, 7, T=0.9, mask="drop5", seed=11))
+    base = _gpu(kd, x, 0.9, 300)
+    again = _gpu(kd, x, 0.9, 300)
+    for k in ("lse", "dH", "dW"):
+        assert np.array_equal(base[k], again[k]), f"rerun changed {k}"
+    assert base["loss"] == again["loss"]
+    for chunk in (1, 64, 128, 299):
+        r = _gpu(kd, x, 0.9, chunk)
+        assert r["loss"] == base["loss"] and np.array_equal(r["lse"], base["lse"])
+        assert np.array_equal(r["dH"], base["dH"]), f"dH depends on chunk={chunk}"
+        assert _rfro(r["dW"], base["dW"]) <= 1e-5, f"dW chunk={chunk}"
+
+
+def test_duplicate_teacher_indices(kd):
+    x = workloads.make_inputs(_cfg(200, 64, 700, 6, seed=5))
+    x["topk_idx"][:, 3] = x["topk_idx"][:, 0]
+    x["topk_idx"][::7, 5] = x["topk_idx"][::7, 0]
+    ref = _oracle(x, 1.0)
+    got = _gpu(kd, x, 1.0, 64)
+    _assert_parity(got, ref, "duplicates")
+
+
+def test_zero_mask_sum(kd):
+    x = workloads.make_inputs(_cfg(130, 64, 600, 4, seed=6))
+    x["mask"].zero_()
+    ref = _oracle(x, 1.0)
+    got = _gpu(kd, x, 1.0, 64)
+    assert got["loss"] == 0.0 and ref["loss"] == 0.0
+    assert np.all(got["dH"] == 0.0) and np.all(got["dW"] == 0.0)
+    assert np.max(np.abs(got["lse"] - ref["lse"])) <= LSE_ATOL
+
+
+def test_neg_inf_teacher_logit(kd):
+    x = workloads.make_inputs(_cfg(140, 64, 900, 8, seed=7))
+    x["topk_logit"][::3, -1] = -math.inf
+    ref = _oracle(x, 1.0)
+    got = _gpu(kd, x, 1.0, 64)
+    _assert_parity(got, ref, "-inf logits")
+
+
+def test_accumulate_dW(kd):
+    x = workloads.make_inputs(_cfg(200, 64, 700, 6, seed=8))
+    g = _to_dev(x)
+    ws = kd.alloc_workspace(200, 64, 700, 6, 64, "cuda")
+    _, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws)
+    dW0 = torch.randn(700, 64, device="cuda")
+    _, dW = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, lse,
+                        dW=dW0.clone(), accumulate_dW=True, workspace=ws)
+    _, dW1 = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, lse,
+                         workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.allclose(dW, dW0 + dW1, rtol=0, atol=1e-6)
+
+
+def test_empty_input(kd):
+    H = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    W = torch.randn(100, 64, device="cuda").to(torch.bfloat16)
+    idx = torch.empty(0, 4, dtype=torch.int32, device="cuda")
+    lg = torch.empty(0, 4, dtype=torch.float32, device="cuda")
+    loss, lse = kd.forward(H, W, idx, lg, None, 1.0, 64)
+    dH, dW = kd.backward(H, W, idx, lg, None, 1.0, 64, lse)
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0 and lse.numel() == 0 and dH.numel() == 0
+    assert torch.count_nonzero(dW).item() == 0
+
+
+def test_bad_index_is_reported(kd):
+    x = workloads.make_inputs(_cfg(64, 64, 500, 4, seed=9))
+    x["topk_idx"][3, 1] = 500
+    x["topk_idx"][9, 0] = -2
+    g = _to_dev(x)
+    ws = kd.alloc_workspace(64, 64, 500, 4, 64, "cuda")
+    kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws)
+    st, nbad = kd.check(ws)
+    assert st == 5 and nbad == 2
+    # the workspace status is per call: a clean call clears it
+    g["topk_idx"][3, 1] = 1
+    g["topk_idx"][9, 0] = 2
+    kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws)
+    assert kd.check(ws) == (0, 0)
+
+
+def test_autograd_wrapper(kd):
+    x = workloads.make_inputs(_cfg(256, 128, 1000, 8, seed=10))
+    g = _to_dev(x)
+    H = g["H"].clone().requires_grad_(True)
+    W = g["W"].clone().requires_grad_(True)
+    loss = kd.kd_topk_kl_loss(H, W, g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 128)
+    (3.0 * loss).backward()
+    ref = _oracle(x, 1.0, grad=3.0)
+    assert abs(loss.item() - ref["loss"]) / ref["loss"] <= LOSS_RTOL
+    assert _rfro(H.grad.float().cpu().double().numpy(), ref["dH"]) <= GRAD_RFRO
+    assert _rfro(W.grad.float().cpu().double().numpy(), ref["dW"]) <= GRAD_RFRO
