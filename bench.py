@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the fused chunked top-K KL loss (forward + backward) on B200.
+
+One step = one forward and one backward pass of the whole path over one
+batch of synthetic inputs (teacher-cache preparation, logits + online
+log-sum-exp + teacher gather, lse merge and loss, then per chunk the logit
+recompute into dZ, dH = dZ W and dW += dZ^T H).  Inputs are resident in HBM
+before the timed region starts.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--N TOKENS]
+  python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host
+
+For N > 1 it runs under torch.distributed.run, one process per GPU; each
+rank computes an independent replica (the path has no exchange step), the
+timed region is bracketed by barriers, and the time is the maximum over
+ranks.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused top-K KL fwd+bwd tokens/s, TFLOP/s (% bf16 tensor peak); peak HBM GiB"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_CONFIG = 3
+L2_BYTES = 126 * 2**20
+KERNEL_SOURCES = ["kd_gemm.cuh", "kd_ptx.cuh", "kd_schedule.h", "kd_small_kernels.cuh", "kd_topk_kl.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_fwd_traffic.txt")
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "chunked_top_kl_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per launch of the forward GEMM from the committed ncu
+    summary, if it was taken on this workload and on the current sources."""
+    try:
+        kv = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_hash") != kernel_source_hash() or kv.get("workload") != workload:
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(impl: str):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and impl == "cuda":
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def launches_per_step(N: int, chunk: int) -> int:
+    """Kernels this library launches for one forward + one backward call:
+    forward = teacher prep, logits/lse GEMM, lse merge, finalize;
+    backward = teacher prep, finalize, and per chunk dZ, dH and dW GEMMs."""
+    if N == 0:
+        return 0
+    return 4 + 2 + 3 * math.ceil(N / chunk)
+
+
+def blas_threads() -> int:
+    try:
+        import numpy  # noqa: F401  (load the BLAS so threadpoolctl can see it)
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(x, cfg, n_tokens: int):
+    """Time the fp64 oracle (as it stands) on the first n_tokens tokens of the
+    workload: forward + backward of those tokens against the full W."""
+    import oracle
+    sub = {k: (v[:n_tokens] if k != "W" else v) for k, v in x.items()}
+    t0 = time.perf_counter()
+    oracle.kd_topk_kl(sub["H"], sub["W"], sub["topk_idx"], sub["topk_logit"], sub["mask"], cfg.T)
+    return time.perf_counter() - t0
+
+
+def sample_tokens(cfg, flop_budget: float) -> int:
+    return int(max(1, min(cfg.N, round(flop_budget / (8.0 * cfg.d * cfg.V)))))
+
+
+# ---------------------------------------------------------------- arms
+
+def run_reference(args, cfg, world, rank):
+    if rank != 0:
+        return 0
+    x = workloads.make_inputs(cfg)
+    n = sample_tokens(cfg, args.ref_flops)
+    for _ in range(args.warmup):
+        oracle_sample(x, cfg, n)
+    times = [oracle_sample(x, cfg, n) for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    cores = blas_threads()
+    flops = 8.0 * n * cfg.d * cfg.V * args.steps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "tflops": flops / total / 1e12,
+        "config": config_block(cfg, 1),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {n} of {cfg.N} tokens per step (full W, fwd+bwd, fp64)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, world):
+    return {"workload": cfg.name, "N": cfg.N, "d": cfg.d, "V": cfg.V, "K": cfg.K, "T": cfg.T,
+            "chunk": cfg.chunk, "seed": cfg.seed, "mask": cfg.mask, "teacher": cfg.teacher,
+            "global_batch": cfg.N * world, "seq_len": cfg.N,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (W is %.2f GB > 126 MB L2); no flush" % (2 * cfg.V * cfg.d / 1e9)}
+
+
+def run_cuda(args, cfg, world, rank, local):
+    import chunked_top_kl_b200 as kd
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    rcfg = cfg if rank == 0 else cfg.__class__(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
+    x = workloads.make_inputs(rcfg)
+    N, d, V, K, T, chunk = cfg.N, cfg.d, cfg.V, cfg.K, cfg.T, cfg.chunk
+
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_mem = torch.cuda.memory_allocated(dev)
+    g = {k: v.to(dev) for k, v in x.items()}
+    ws = kd.alloc_workspace(N, d, V, K, chunk, dev)
+    dH = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, workspace=ws)
+        kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, lse,
+                    workspace=ws, dH=dH, dW=dW)
+        return loss
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, nbad = kd.check(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {kd.kd_status_string(st)}")
+    peak_gib = (torch.cuda.max_memory_allocated(dev) - base_mem) / 2**30
+    ws_gib = ws.numel() / 2**30
+
+    # ---- kernel-only timed region (inputs resident in HBM)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local) if not args.no_clocks else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, workspace=ws)
+        ev[i][1].record(stream)
+        kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, lse,
+                    workspace=ws, dH=dH, dW=dW)
+        ev[i][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms_local = start.elapsed_time(end)
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    ms = reduce_max(ms_local, world, dev)
+    st, _ = kd.check(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {kd.kd_status_string(st)}")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.pin_memory() for k, v in x.items()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        loss_host = torch.empty((), dtype=torch.float32).pin_memory()
+        for _ in range(max(1, args.warmup)):
+            for k in g:
+                g[k].copy_(host[k], non_blocking=True)
+            loss = step()
+            loss_host.copy_(loss, non_blocking=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        s2 = torch.cuda.Event(enable_timing=True)
+        e2 = torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            for k in g:
+                g[k].copy_(host[k], non_blocking=True)
+            loss = step()
+            loss_host.copy_(loss, non_blocking=True)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = reduce_max(s2.elapsed_time(e2), world, dev)
+        e2e = {"value": N * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(loss_host.element_size()),
+               "ms_per_step": e2e_ms / args.steps}
+
+    if rank != 0:
+        return 0
+
+    peaks, peaks_src = load_peaks()
+    ms_step = ms / args.steps
+    flops_step = 8.0 * N * d * V
+    tflops = flops_step * world / (ms_step / 1e3) / 1e12
+    # Roofline of the single longest launch: the forward GEMM (logits + online
+    # lse + teacher gather).  Its call also holds three tiny CUDA-core kernels
+    # (teacher prep, lse merge, finalize), which are counted in its time.
+    fwd_avg = sum(fwd_ms) / len(fwd_ms)
+    fwd_ach = 2.0 * N * d * V / (fwd_avg / 1e3) / 1e12
+    bwd_avg = sum(bwd_ms) / len(bwd_ms)
+    peak_sus = peaks["bf16_tflops_sustained"]
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        n = sample_tokens(cfg, args.cpu_flops)
+        t = oracle_sample(x, cfg, n)
+        cpu = {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {n} of {N} tokens (full W), fwd+bwd in fp64, one run of {t:.1f} s"}
+    line = {
+        "metric": METRIC, "value": N * world * args.steps / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; H~N(0,1), W~N(0,0.02^2) bf16, Zipf-shaped top-K teacher cache)",
+        "tflops": tflops,
+        "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
+        "pct_bf16_peak_sustained": tflops / world / peak_sus,
+        "peak_hbm_gib": peak_gib, "workspace_gib": ws_gib,
+        "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
+        "config": config_block(cfg, world),
+        "clocks": clocks,
+        "gpu_launches": launches_per_step(N, chunk) * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel<EpiFwd> (forward logits/lse/gather)",
+                     "achieved": fwd_ach, "peak": peak_sus, "unit": "TFLOP/s", "frac": fwd_ach / peak_sus,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks_src})",
+                     "frac_of_burst": fwd_ach / peaks["bf16_tflops"],
+                     "flops_per_launch": 2.0 * N * d * V,
+                     "traffic": committed_traffic(cfg.name)},
+        "roofline_step": {"bound": "tensor", "achieved": tflops / world, "peak": peak_sus,
+                          "unit": "TFLOP/s", "frac": tflops / world / peak_sus,
+                          "flops_per_step": flops_step},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
+    ap.add_argument("--N", type=int, default=None, help="override the token count (config 4 sweep)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-flops", type=float, default=4e12, help="oracle work for cpu_baseline")
+    ap.add_argument("--ref-flops", type=float, default=1.2e12, help="oracle work per reference step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = workloads.get_config(args.config, args.N)
+    world, rank, local = dist_setup(args.impl)
+    if world != args.gpus and args.impl == "cuda":
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, cfg, world, rank)
+        return run_cuda(args, cfg, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "cuda":
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())
