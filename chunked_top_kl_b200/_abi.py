@@ -26,6 +26,7 @@ EXPORTS = (
     "kd_topk_kl_forward",
     "kd_topk_kl_backward",
     "kd_topk_kl_check",
+    "kd_topk_kl_forward_noalloc",
 )
 
 _lib = None
@@ -51,6 +52,8 @@ def load() -> ctypes.CDLL:
         lib.kd_topk_kl_backward.restype = i32
         lib.kd_topk_kl_check.argtypes = [p, p, ctypes.POINTER(i64)]
         lib.kd_topk_kl_check.restype = i32
+        lib.kd_topk_kl_forward_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, p, p, p]
+        lib.kd_topk_kl_forward_noalloc.restype = i32
         _lib = lib
     return _lib
 
@@ -86,3 +89,11 @@ def kd_topk_kl_check(workspace, stream) -> tuple[int, int]:
     n = ctypes.c_int64(0)
     st = int(load().kd_topk_kl_check(workspace, stream, ctypes.byref(n)))
     return st, int(n.value)
+
+
+def kd_topk_kl_forward_noalloc(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, loss, lse,
+                               stream) -> int:
+    """Forward pass on the library's built-in 16 MiB scratch array, for
+    callers that cannot allocate device memory (see the C header)."""
+    return int(load().kd_topk_kl_forward_noalloc(H, W, topk_idx, topk_logit, mask, N, d, V, K, T,
+                                                 loss, lse, stream))

@@ -347,3 +347,50 @@ int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_cou
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- forward without a workspace
+//
+// Some callers cannot allocate device memory at the point where they need
+// the loss: code running under a runtime that owns every byte of device
+// memory (a serving process that reserves HBM up front and hands out only
+// fixed buffers), plug-ins called while their host framework holds its
+// allocator lock, and latency-critical loops for which cudaMalloc's implicit
+// synchronisation is not acceptable.  For them the forward pass can run on a
+// fixed scratch array that lives in this library's own device image.
+//
+// The array is kNoAllocScratchBytes (16 MiB) on every device that loads the
+// library and stays allocated until the process exits.  In host code the
+// symbol is only a host-side stand-in, so its device address is looked up
+// with cudaGetSymbolAddress once per device, on that device's first call.
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+void* g_noalloc_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+extern "C" int kd_topk_kl_forward_noalloc(const void* H, const void* W, const int32_t* topk_idx,
+                                          const float* topk_logit, const float* mask, int64_t N,
+                                          int64_t d, int64_t V, int64_t K, float T, float* loss,
+                                          float* lse, void* stream) {
+  int st = check_shapes(N, d, V, K, T, 1);
+  if (st != KD_OK) return st;
+  // The forward pass needs no dZ chunk, so the smallest chunk keeps the
+  // layout (and the size limit) to the prepared teacher cache, the per-token
+  // partial log-sum-exp state and the status words.
+  if (make_layout(N, V, K, 1).total > kNoAllocScratchBytes) return KD_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KD_ERR_UNSUPPORTED;
+  if (!g_noalloc_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KD_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev] = p;
+  }
+  // Every word the forward pass reads from the scratch is written earlier in
+  // the same call (the status words are cleared at its start), so nothing
+  // left over from a previous call is ever used.
+  return kd_topk_kl_forward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, 1, loss, lse,
+                            g_noalloc_scratch_ptr[dev], kNoAllocScratchBytes, stream);
+}

@@ -25,9 +25,11 @@
  * probabilities at that column (the loss keeps the per-slot sum).
  *
  * Conventions shared by every entry point:
- *  - All array pointers are DEVICE pointers owned by the caller.  The
- *    library never allocates device or host memory and keeps no state
- *    between calls except a per-device, per-kernel attribute cache.
+ *  - All array pointers are DEVICE pointers owned by the caller.  No call
+ *    allocates device or host memory.  The library keeps no state between
+ *    calls except a per-device, per-kernel attribute cache and, for
+ *    kd_topk_kl_forward_noalloc only, a fixed scratch array in its own
+ *    device image.
  *  - Layouts are dense row-major: H bf16 [N][d], W bf16 [V][d],
  *    topk_idx int32 [N][K], topk_logit fp32 [N][K], mask fp32 [N],
  *    lse fp32 [N], dH bf16 [N][d], dW fp32 [V][d].  bf16 is IEEE bfloat16
@@ -106,6 +108,36 @@ int kd_topk_kl_backward(const void* H, const void* W,
                         const float* lse, const float* grad_loss,
                         void* dH, float* dW, int accumulate_dW,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward pass for callers that cannot allocate device memory.  The paper
+ * has no counterpart to this entry point; it exists for callers such as a
+ * runtime that owns all device memory and hands out only fixed buffers, a
+ * plug-in called while its host framework holds its allocator lock, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit
+ * synchronisation.
+ *
+ * Same inputs and outputs as kd_topk_kl_forward (no chunk, no workspace).
+ * Instead of a caller workspace it uses a 16 MiB scratch array compiled into
+ * the library: every device that loads the library holds those 16 MiB until
+ * the process exits.  It allocates nothing itself (no cudaMalloc, no
+ * cudaFree, no allocating library call).
+ *  - Size limit: kd_topk_kl_workspace_size(N, d, V, K, 1) must not exceed
+ *    16 MiB (about 1 KiB per token at K = 100, so up to roughly 16,000
+ *    tokens); larger sizes return KD_ERR_WORKSPACE and enqueue nothing.
+ *  - The first call on each device looks up the scratch array's device
+ *    address (cudaGetSymbolAddress) with that device current; make that
+ *    first call before any stream capture begins.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    the pass clears its status words and overwrites everything else it
+ *    reads before reading it.  Calls that overlap on the GPU (different
+ *    streams, or different host threads) race on the array and must not be
+ *    issued.  Device-side status (bad teacher indices) is not reported
+ *    through kd_topk_kl_check for this entry point. */
+int kd_topk_kl_forward_noalloc(const void* H, const void* W,
+                               const int32_t* topk_idx, const float* topk_logit,
+                               const float* mask,
+                               int64_t N, int64_t d, int64_t V, int64_t K, float T,
+                               float* loss, float* lse, void* stream);
 
 /* Synchronises `stream`, then reads the device-side status words that the
  * last forward or backward call on this workspace wrote.  Returns KD_OK,
