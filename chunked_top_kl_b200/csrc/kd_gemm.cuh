@@ -25,17 +25,29 @@
 
 namespace kd {
 
-constexpr int BM = 128;          // tile rows (TMEM lanes)
+constexpr int BM = 128;          // accumulator rows per CTA (TMEM lanes)
 constexpr int BN = 256;          // tile columns (TMEM columns per accumulator)
 constexpr int BK = 64;           // bf16 elements per 128-byte swizzle row
 constexpr int UMMA_K = 16;       // K of one tcgen05.mma kind::f16
-constexpr int STAGES = 4;
-constexpr int A_STAGE_BYTES = BM * BK * 2;
-constexpr int B_STAGE_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int GEMM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+// Per-variant tile geometry.  PAIR = false: one CTA computes a 128 x 256 tile
+// (A 128 rows, B 256 rows per stage).  PAIR = true: a cluster of two CTAs
+// computes a 256 x 256 tile with cta_group::2 MMAs; each CTA stages its own
+// 128 rows of A and 128 rows of B, holds its 128 accumulator rows in its own
+// tensor memory, and the pair leader issues the MMAs.
+template <bool PAIR>
+struct Geo {
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;          // B rows staged per CTA
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // per CTA
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // per stage, whole tile
+};
 
 struct GemmArgs {
   Raster raster;
@@ -50,14 +62,18 @@ struct GemmArgs {
 //           8-row groups 1024 B apart (SBO), 128-byte swizzled.
 //  MN-major: rows/64 boxes {64, BK} at (row + 64 i, k).  Each box is BK
 //           K-rows of 128 B (64 MN elements); boxes are BK*128 B apart (LBO).
-template <bool MN_MAJOR, int ROWS>
+template <bool MN_MAJOR, int ROWS, bool PAIR>
 __device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* tm, int row, int k,
                                              uint32_t bar) {
   if constexpr (!MN_MAJOR) {
-    tma_load_2d(dst, tm, k, row, bar);
+    if constexpr (PAIR) tma_load_2d_pair(dst, tm, k, row, bar);
+    else tma_load_2d(dst, tm, k, row, bar);
   } else {
 #pragma unroll
-    for (int i = 0; i < ROWS / 64; ++i) tma_load_2d(dst + i * (BK * 128), tm, row + 64 * i, k, bar);
+    for (int i = 0; i < ROWS / 64; ++i) {
+      if constexpr (PAIR) tma_load_2d_pair(dst + i * (BK * 128), tm, row + 64 * i, k, bar);
+      else tma_load_2d(dst + i * (BK * 128), tm, row + 64 * i, k, bar);
+    }
   }
 }
 
@@ -73,15 +89,17 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
   }
 }
 
-template <class Epi, bool A_MN, bool B_MN>
+template <class Epi, bool A_MN, bool B_MN, bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const GemmArgs args, const typename Epi::Params ep) {
+  using G = Geo<PAIR>;
+  constexpr int STAGES = G::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * G::STAGE_BYTES);
   const uint32_t bar_base = smem_u32(bars);
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
@@ -93,6 +111,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const Raster& R = args.raster;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;       // CTA within the pair
+  const int group = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int ngroups = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  // Barriers that the pair leader owns: stage-full (TMA bytes of both CTAs)
+  // and accumulator-empty (epilogue threads of both CTAs).
+  auto leader = [&](uint32_t a) { return PAIR ? mapa_shared(a, 0) : a; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -101,7 +125,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4 * 32);
+      mbar_init(tempty_bar(a), (PAIR ? 2 : 1) * 4 * 32);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -111,45 +135,53 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   bool failed = false;
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (every CTA)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int u = blockIdx.x; u < R.num_units && !failed; u += gridDim.x) {
+      for (int u = group; u < R.num_units && !failed; u += ngroups) {
         int m, split, n0, n1;
         decode_unit(R, u, m, split, n0, n1);
         for (int n = n0; n < n1 && !failed; ++n) {
           for (int kb = 0; kb < args.num_kb; ++kb) {
             if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag)) { failed = true; break; }
-            const uint32_t sa = sbase + stage * STAGE_BYTES;
-            const uint32_t sb = sa + A_STAGE_BYTES;
-            mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-            load_operand<A_MN, BM>(sa, &tmA, args.a_row0 + m * BM, args.a_k0 + kb * BK, full_bar(stage));
-            load_operand<B_MN, BN>(sb, &tmB, args.b_row0 + n * BN, args.b_k0 + kb * BK, full_bar(stage));
+            const uint32_t sa = sbase + stage * G::STAGE_BYTES;
+            const uint32_t sb = sa + G::A_BYTES;
+            const uint32_t fb = leader(full_bar(stage));
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), G::TX_BYTES);
+            load_operand<A_MN, BM, PAIR>(sa, &tmA, args.a_row0 + m * G::TILE_M + (int)rank * BM,
+                                         args.a_k0 + kb * BK, fb);
+            load_operand<B_MN, G::B_ROWS, PAIR>(sb, &tmB, args.b_row0 + n * BN + (int)rank * G::B_ROWS,
+                                                args.b_k0 + kb * BK, fb);
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+    // ------------------------------------------------------------ MMA issuer (pair leader)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(G::TILE_M, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = blockIdx.x; u < R.num_units && !failed; u += gridDim.x) {
+      for (int u = group; u < R.num_units && !failed; u += ngroups) {
         int m, split, n0, n1;
         decode_unit(R, u, m, split, n0, n1);
         for (int n = n0; n < n1 && !failed; ++n) {
@@ -159,48 +191,53 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           for (int kb = 0; kb < args.num_kb; ++kb) {
             if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag)) { failed = true; break; }
             tc_fence_after();
-            const uint32_t sa = sbase + stage * STAGE_BYTES;
-            const uint32_t sb = sa + A_STAGE_BYTES;
+            const uint32_t sa = sbase + stage * G::STAGE_BYTES;
+            const uint32_t sb = sa + G::A_BYTES;
 #pragma unroll
             for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-              tc_mma_bf16(d_tmem, operand_desc<A_MN>(sa, kk), operand_desc<B_MN>(sb, kk), idesc,
-                          (kb | kk) != 0 ? 1u : 0u);
+              const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+              if constexpr (PAIR)
+                tc_mma_bf16_pair(d_tmem, operand_desc<A_MN>(sa, kk), operand_desc<B_MN>(sb, kk), idesc, accum);
+              else
+                tc_mma_bf16(d_tmem, operand_desc<A_MN>(sa, kk), operand_desc<B_MN>(sb, kk), idesc, accum);
             }
-            tc_commit(empty_bar(stage));
+            if constexpr (PAIR) tc_commit_pair_mc(empty_bar(stage), 0x3); else tc_commit(empty_bar(stage));
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
           if (failed) break;
-          tc_commit(tfull_bar(acc));
+          if constexpr (PAIR) tc_commit_pair_mc(tfull_bar(acc), 0x3); else tc_commit(tfull_bar(acc));
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
         }
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (every CTA)
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int row = q * 32 + lane;          // tile row owned by this thread
+    const int row = (int)rank * BM + q * 32 + lane;   // row of the tile owned by this thread
     const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
     Epi epi;
-    for (int u = blockIdx.x; u < R.num_units && !failed; u += gridDim.x) {
+    for (int u = group; u < R.num_units && !failed; u += ngroups) {
       int m, split, n0, n1;
       decode_unit(R, u, m, split, n0, n1);
-      epi.begin_unit(ep, m, split, n0, row);
+      const int grow = m * G::TILE_M + row;
+      epi.begin_unit(ep, grow, split, n0);
       for (int n = n0; n < n1; ++n) {
         // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes.
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag));
         if (!ok) { failed = true; break; }
         tc_fence_after();
-        epi.tile(ep, m, n, row, lane_addr + acc * BN);
+        epi.tile(ep, grow, n, lane_addr + acc * BN);
         tc_fence_before();
-        mbar_arrive(tempty_bar(acc));
+        if constexpr (PAIR) mbar_arrive_cluster(leader(tempty_bar(acc)));
+        else mbar_arrive(tempty_bar(acc));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       if (failed) break;
-      epi.end_unit(ep, m, split, row);
+      epi.end_unit(ep, grow, split);
     }
   }
 
@@ -213,17 +250,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (*abort_flag) {
     // Let asynchronous copies and MMAs that were already issued land before
     // the CTA releases its shared and tensor memory.
-    if (warp == 1 && lane == 0) {
-      const uint32_t drain = tfull_bar(0);
-      tc_commit(drain);
-    }
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 2000000ull) { }
     __syncthreads();
   }
+  // Neither CTA of a pair may release its memory while the leader's MMAs can
+  // still read the peer's shared memory or write its tensor memory.
+  if constexpr (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -255,8 +292,8 @@ struct EpiFwd {
   const int32_t* trow;
   const float* prow;
 
-  __device__ __forceinline__ void begin_unit(const Params& P, int m, int, int n0, int row) {
-    grow = m * BM + row;
+  __device__ __forceinline__ void begin_unit(const Params& P, int grow_, int, int n0) {
+    grow = grow_;
     mrun = -INFINITY;
     srun = 0.f;
     grun = 0.f;
@@ -271,7 +308,7 @@ struct EpiFwd {
     }
   }
 
-  __device__ __forceinline__ void tile(const Params& P, int, int n, int, uint32_t taddr) {
+  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr) {
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       float v[32];
@@ -307,7 +344,7 @@ struct EpiFwd {
     }
   }
 
-  __device__ __forceinline__ void end_unit(const Params& P, int, int split, int) {
+  __device__ __forceinline__ void end_unit(const Params& P, int, int split) {
     if (grow < P.N) {
       const size_t o = (size_t)split * P.N + grow;
       P.part_m[o] = mrun;
@@ -337,11 +374,10 @@ struct EpiDz {
     const float* cscale;   // device scalar g / sum(mask)
     __nv_bfloat16* dz;
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, int) {}
-  __device__ __forceinline__ void end_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int m, int n, int row, uint32_t taddr) {
-    const int r = m * BM + row;
+  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr) {
     const bool valid = r < P.rows_valid;
     const int grow = P.row0 + r;
     float L = 0.f, c = 0.f;
@@ -403,11 +439,10 @@ struct EpiDh {
     int rows_valid, row0, d;
     __nv_bfloat16* dH;
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, int) {}
-  __device__ __forceinline__ void end_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int m, int n, int row, uint32_t taddr) {
-    const int r = m * BM + row;
+  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr) {
     const bool valid = r < P.rows_valid;
     __nv_bfloat16* out = P.dH + (size_t)(P.row0 + r) * P.d;
 #pragma unroll 1
@@ -439,11 +474,10 @@ struct EpiDw {
     int rows_valid, d, accumulate;
     float* dW;
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, int) {}
-  __device__ __forceinline__ void end_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int m, int n, int row, uint32_t taddr) {
-    const int r = m * BM + row;
+  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr) {
     const bool valid = r < P.rows_valid;
     float* out = P.dW + (size_t)r * P.d;
 #pragma unroll 1

@@ -111,6 +111,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 
 struct DevInfo {
   int sms = 0;
+  int pair_groups = 0;          // co-resident CTA pairs of the GEMM kernel
   bool attr_set[8] = {};
 };
 DevInfo g_dev[kMaxDevices];
@@ -125,20 +126,72 @@ int device_sms(int dev) {
   return g_dev[dev].sms;
 }
 
-template <class Epi, bool A_MN, bool B_MN>
-cudaError_t launch_gemm(int slot, int dev, int grid, const CUtensorMap& ta, const CUtensorMap& tb,
+// All GEMMs run as CTA pairs (cta_group::2, 256 x 256 tiles).
+constexpr bool kPair = true;
+using GeoP = Geo<kPair>;
+
+template <class Epi, bool A_MN, bool B_MN, bool PAIR>
+cudaError_t launch_gemm(int slot, int dev, int groups, const CUtensorMap& ta, const CUtensorMap& tb,
                         const GemmArgs& args, const typename Epi::Params& ep, cudaStream_t s) {
-  auto kern = gemm_tc_kernel<Epi, A_MN, B_MN>;
+  using G = Geo<PAIR>;
+  auto kern = gemm_tc_kernel<Epi, A_MN, B_MN, PAIR>;
   if (dev >= 0 && dev < kMaxDevices && !g_dev[dev].attr_set[slot]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    if (PAIR) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+      (void)e;
+    }
     g_dev[dev].attr_set[slot] = true;
   }
-  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, args, ep);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(groups * (PAIR ? 2 : 1)), 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = G::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args, ep);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-inline int grid_for(const Raster& r, int sms) { return r.num_units < sms ? r.num_units : sms; }
+// Work groups (CTAs, or CTA pairs) that can be resident at once: one per SM,
+// or per pair of SMs that the hardware can co-schedule as a cluster.
+int resident_groups(int dev) {
+  const int sms = device_sms(dev);
+  if (!kPair) return sms;
+  if (dev < 0 || dev >= kMaxDevices) return sms / 2;
+  if (!g_dev[dev].pair_groups) {
+    auto kern = gemm_tc_kernel<EpiDz, false, false, true>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GeoP::SMEM_BYTES);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sms, 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = GeoP::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sms / 2;
+    }
+    g_dev[dev].pair_groups = n < sms / 2 ? n : sms / 2;
+  }
+  return g_dev[dev].pair_groups;
+}
+
+inline int grid_for(const Raster& r, int groups) { return r.num_units < groups ? r.num_units : groups; }
 
 int common_checks(const void* H, const void* W, const int32_t* idx, const float* logit,
                   int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
@@ -210,11 +263,11 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
 
   CUtensorMap tmH, tmW;
-  if (!make_map(&tmH, H, d, N, d, BK, BM) || !make_map(&tmW, W, d, V, d, BK, BN))
+  if (!make_map(&tmH, H, d, N, d, BK, BM) || !make_map(&tmW, W, d, V, d, BK, GeoP::B_ROWS))
     return KD_ERR_CUDA;
-  const int sms = device_sms(dev);
+  const int groups = resident_groups(dev);
   GemmArgs a{};
-  a.raster = forward_raster(ceil_div(N, BM), ceil_div(V, BN), sms);
+  a.raster = forward_raster(ceil_div(N, GeoP::TILE_M), ceil_div(V, BN), groups);
   a.num_kb = (int)ceil_div(d, BK);
   a.status = status;
   EpiFwd::Params ep{};
@@ -226,7 +279,7 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   ep.part_m = at<float>(workspace, L.off_pm);
   ep.part_s = at<float>(workspace, L.off_ps);
   ep.part_g = at<float>(workspace, L.off_pg);
-  if (launch_gemm<EpiFwd, false, false>(0, dev, grid_for(a.raster, sms), tmH, tmW, a, ep, s) != cudaSuccess)
+  if (launch_gemm<EpiFwd, false, false, kPair>(0, dev, grid_for(a.raster, groups), tmH, tmW, a, ep, s) != cudaSuccess)
     return KD_ERR_CUDA;
 
   lse_merge_kernel<<<(unsigned)L.n_merge_blocks, kMergeThreads, 0, s>>>(
@@ -273,10 +326,10 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
 
   CUtensorMap tmHk, tmWk, tmWmn, tmHmn;
-  if (!make_map(&tmHk, H, d, N, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, BN) ||
+  if (!make_map(&tmHk, H, d, N, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, GeoP::B_ROWS) ||
       !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, H, d, N, d, 64, BK))
     return KD_ERR_CUDA;
-  const int sms = device_sms(dev);
+  const int groups = resident_groups(dev);
 
   for (int64_t c0 = 0; c0 < N; c0 += chunk) {
     const int64_t Cc = (N - c0 < chunk) ? (N - c0) : chunk;
@@ -286,7 +339,7 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
 
     // dZ for the chunk: recompute z = H W^T tile by tile.
     GemmArgs a3{};
-    a3.raster = tile_raster(ceil_div(Cc, BM), ceil_div(V, BN), true);
+    a3.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), true);
     a3.num_kb = (int)ceil_div(d, BK);
     a3.a_row0 = (int)c0;
     a3.status = status;
@@ -302,12 +355,12 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     e3.mask = mask;
     e3.cscale = cscale;
     e3.dz = dz;
-    if (launch_gemm<EpiDz, false, false>(1, dev, grid_for(a3.raster, sms), tmHk, tmWk, a3, e3, s) != cudaSuccess)
+    if (launch_gemm<EpiDz, false, false, kPair>(1, dev, grid_for(a3.raster, groups), tmHk, tmWk, a3, e3, s) != cudaSuccess)
       return KD_ERR_CUDA;
 
     // dH[chunk] = dZ W   (A = dZ, K-major over V; B = W, MN-major over d).
     GemmArgs a4{};
-    a4.raster = tile_raster(ceil_div(Cc, BM), ceil_div(d, BN), true);
+    a4.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), true);
     a4.num_kb = (int)ceil_div(V, BK);
     a4.status = status;
     EpiDh::Params e4{};
@@ -315,12 +368,12 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     e4.row0 = (int)c0;
     e4.d = (int)d;
     e4.dH = static_cast<__nv_bfloat16*>(dH);
-    if (launch_gemm<EpiDh, false, true>(2, dev, grid_for(a4.raster, sms), tmZk, tmWmn, a4, e4, s) != cudaSuccess)
+    if (launch_gemm<EpiDh, false, true, kPair>(2, dev, grid_for(a4.raster, groups), tmZk, tmWmn, a4, e4, s) != cudaSuccess)
       return KD_ERR_CUDA;
 
     // dW (+)= dZ^T H[chunk]   (A = dZ^T, MN-major over V; B = H, MN-major over d).
     GemmArgs a5{};
-    a5.raster = tile_raster(ceil_div(V, BM), ceil_div(d, BN), false);
+    a5.raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
     a5.num_kb = (int)ceil_div(Cc, BK);
     a5.b_k0 = (int)c0;
     a5.status = status;
@@ -329,7 +382,7 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     e5.d = (int)d;
     e5.accumulate = (accumulate_dW || c0 > 0) ? 1 : 0;
     e5.dW = dW;
-    if (launch_gemm<EpiDw, true, true>(3, dev, grid_for(a5.raster, sms), tmZmn, tmHmn, a5, e5, s) != cudaSuccess)
+    if (launch_gemm<EpiDw, true, true, kPair>(3, dev, grid_for(a5.raster, groups), tmZmn, tmHmn, a5, e5, s) != cudaSuccess)
       return KD_ERR_CUDA;
   }
   return KD_OK;
