@@ -45,7 +45,8 @@ struct Geo {
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // per CTA
   static constexpr int STAGES = PAIR ? 6 : 4;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int STAGING_BYTES = 2 * BM * 128;           // two 128-row x 128-byte store buffers
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // per stage, whole tile
 };
 
@@ -89,17 +90,53 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int kk) {
   }
 }
 
+// What an epilogue thread needs to write its tile through shared memory and
+// TMA: two 16 KB staging buffers used alternately, the thread's row in the
+// CTA's 128-row slab, the slab's first output row, and whether this thread
+// issues the bulk copies (one thread of the 128).
+struct EpiCtx {
+  uint32_t stage[2];
+  int rr;
+  int row_base;
+  bool issuer;
+  uint32_t seq;
+};
+
+// Writes one 128-byte segment per thread (its row) into the next staging
+// buffer with the 128-byte swizzle, then one thread stores (or adds) the
+// 128-row box to global memory at (x, y) with TMA.
+__device__ __forceinline__ void stage_store(EpiCtx& cx, const CUtensorMap* tm, int x, int y,
+                                            const uint32_t (&w)[32], bool reduce_add) {
+  const uint32_t buf = cx.stage[cx.seq & 1u];
+  if (cx.issuer && cx.seq >= 2) bulk_wait_read<1>();     // buffer's previous store has read it
+  epilogue_bar_sync(128);
+  const uint32_t rowa = buf + (uint32_t)cx.rr * 128u;
+  const uint32_t sw = (uint32_t)(cx.rr & 7);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    st_shared_v4(rowa + (((uint32_t)k ^ sw) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  fence_proxy_async_shared();
+  epilogue_bar_sync(128);
+  if (cx.issuer) {
+    if (reduce_add) tma_reduce_add_2d(tm, x, y, buf);
+    else tma_store_2d(tm, x, y, buf);
+    bulk_commit();
+  }
+  ++cx.seq;
+}
+
 template <class Epi, bool A_MN, bool B_MN, bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const GemmArgs args, const typename Epi::Params ep) {
+               const GemmArgs args, const __grid_constant__ typename Epi::Params ep) {
   using G = Geo<PAIR>;
   constexpr int STAGES = G::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * G::STAGE_BYTES);
+  const uint32_t staging = sbase + STAGES * G::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * G::STAGE_BYTES + G::STAGING_BYTES);
   const uint32_t bar_base = smem_u32(bars);
   auto full_bar = [&](int s) { return bar_base + 8u * s; };
   auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
@@ -219,17 +256,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int acc = 0;
     uint32_t acc_phase = 0;
     Epi epi;
+    EpiCtx cx;
+    cx.stage[0] = staging;
+    cx.stage[1] = staging + BM * 128;
+    cx.rr = q * 32 + lane;
+    cx.issuer = (threadIdx.x == 64);
+    cx.seq = 0;
     for (int u = group; u < R.num_units && !failed; u += ngroups) {
       int m, split, n0, n1;
       decode_unit(R, u, m, split, n0, n1);
       const int grow = m * G::TILE_M + row;
+      cx.row_base = m * G::TILE_M + (int)rank * BM;
       epi.begin_unit(ep, grow, split, n0);
       for (int n = n0; n < n1; ++n) {
-        // Warp-uniform outcome: tcgen05.ld below needs all 32 lanes.
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag));
+        // One outcome for all 128 epilogue threads: tcgen05.ld needs whole
+        // warps and the store path synchronises the four warps.
+        const bool ok = epilogue_bar_and(128, mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag));
         if (!ok) { failed = true; break; }
         tc_fence_after();
-        epi.tile(ep, grow, n, lane_addr + acc * BN);
+        epi.tile(ep, grow, n, lane_addr + acc * BN, cx);
         tc_fence_before();
         if constexpr (PAIR) mbar_arrive_cluster(leader(tempty_bar(acc)));
         else mbar_arrive(tempty_bar(acc));
@@ -239,6 +284,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (failed) break;
       epi.end_unit(ep, grow, split);
     }
+    if (cx.issuer) bulk_wait<0>();          // every TMA store of this CTA has completed
   }
 
   if (failed) {
@@ -308,7 +354,7 @@ struct EpiFwd {
     }
   }
 
-  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr) {
+  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr, EpiCtx&) {
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       float v[32];
@@ -361,9 +407,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 // Backward, per chunk: dZ = c_n (exp(z - lse_n) - p at the teacher's columns),
 // rounded to bf16 and stored for the chunk's tokens (row-major, ldz columns;
-// columns in [V, ldz) are written as 0).
+// columns in [V, ldz) are written as 0) through shared memory and TMA.
 struct EpiDz {
   struct Params {
+    CUtensorMap tm;        // dZ chunk [rows_valid][ldz] bf16, box {64, 128}, 128-byte swizzle
     int rows_valid;        // tokens in this chunk
     int row0;              // global token index of chunk row 0
     int V, ldz, Kp;
@@ -372,12 +419,11 @@ struct EpiDz {
     const float* lse;
     const float* mask;     // may be null
     const float* cscale;   // device scalar g / sum(mask)
-    __nv_bfloat16* dz;
   };
   __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr) {
+  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr, EpiCtx& cx) {
     const bool valid = r < P.rows_valid;
     const int grow = P.row0 + r;
     float L = 0.f, c = 0.f;
@@ -394,18 +440,20 @@ struct EpiDz {
       nidx = trow[cur];
       np = prow[cur];
     }
-    __nv_bfloat16* out = P.dz + (size_t)r * P.ldz;
 #pragma unroll 1
-    for (int j = 0; j < BN / 32; ++j) {
-      float v[32];
+    for (int j = 0; j < BN / 64; ++j) {
+      float v[64];
+      float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+      float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
       __syncwarp();
-      tmem_ld_32x32b_x32(taddr + j * 32, v);
-      const int c0 = n * BN + j * 32;
+      tmem_ld_32x32b_x32(taddr + j * 64, v0);
+      tmem_ld_32x32b_x32(taddr + j * 64 + 32, v1);
+      const int c0 = n * BN + j * 64;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __expf(v[i] - L);
-      if (nidx < c0 + 32) {
+      for (int i = 0; i < 64; ++i) v[i] = __expf(v[i] - L);
+      if (nidx < c0 + 64) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < 64; ++i) {
           if (c0 + i == nidx) {
             v[i] -= np;
             ++cur;
@@ -414,92 +462,65 @@ struct EpiDz {
           }
         }
       }
+      uint32_t w[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = (c0 + i < P.V) ? c * v[i] : 0.f;
-      if (valid) {
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          if (c0 + 8 * t + 8 <= P.ldz) {
-            uint4 w;
-            w.x = pack_bf16x2(v[8 * t + 0], v[8 * t + 1]);
-            w.y = pack_bf16x2(v[8 * t + 2], v[8 * t + 3]);
-            w.z = pack_bf16x2(v[8 * t + 4], v[8 * t + 5]);
-            w.w = pack_bf16x2(v[8 * t + 6], v[8 * t + 7]);
-            *reinterpret_cast<uint4*>(out + c0 + 8 * t) = w;
-          }
-        }
+      for (int i = 0; i < 32; ++i) {
+        const float a = (c0 + 2 * i < P.V) ? c * v[2 * i] : 0.f;
+        const float b = (c0 + 2 * i + 1 < P.V) ? c * v[2 * i + 1] : 0.f;
+        w[i] = pack_bf16x2(a, b);
       }
+      stage_store(cx, &P.tm, c0, cx.row_base, w, false);
     }
   }
 };
 
-// Backward, per chunk: dH rows of the chunk's tokens, bf16.
+// Backward, per chunk: dH rows of the chunk's tokens, bf16, through shared
+// memory and TMA (the map covers the chunk's rows only).
 struct EpiDh {
   struct Params {
-    int rows_valid, row0, d;
-    __nv_bfloat16* dH;
+    CUtensorMap tm;        // dH rows of the chunk [rows][d] bf16, box {64, 128}, 128-byte swizzle
   };
   __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr) {
-    const bool valid = r < P.rows_valid;
-    __nv_bfloat16* out = P.dH + (size_t)(P.row0 + r) * P.d;
+  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr, EpiCtx& cx) {
 #pragma unroll 1
-    for (int j = 0; j < BN / 32; ++j) {
-      float v[32];
+    for (int j = 0; j < BN / 64; ++j) {
+      float v[64];
+      float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
+      float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
       __syncwarp();
-      tmem_ld_32x32b_x32(taddr + j * 32, v);
-      const int c0 = n * BN + j * 32;
-      if (valid) {
+      tmem_ld_32x32b_x32(taddr + j * 64, v0);
+      tmem_ld_32x32b_x32(taddr + j * 64 + 32, v1);
+      uint32_t w[32];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          if (c0 + 8 * t + 8 <= P.d) {
-            uint4 w;
-            w.x = pack_bf16x2(v[8 * t + 0], v[8 * t + 1]);
-            w.y = pack_bf16x2(v[8 * t + 2], v[8 * t + 3]);
-            w.z = pack_bf16x2(v[8 * t + 4], v[8 * t + 5]);
-            w.w = pack_bf16x2(v[8 * t + 6], v[8 * t + 7]);
-            *reinterpret_cast<uint4*>(out + c0 + 8 * t) = w;
-          }
-        }
-      }
+      for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+      stage_store(cx, &P.tm, n * BN + j * 64, cx.row_base, w, false);
     }
   }
 };
 
-// Backward, per chunk: dW (+)= dZ^T H for 128 vocabulary rows x 256 columns.
+// Backward, per chunk: dW (+)= dZ^T H for 128 vocabulary rows x 256 columns
+// per CTA, fp32, stored (first chunk without accumulation) or added in place
+// by TMA reductions: the memory system does the read-modify-write.
 struct EpiDw {
   struct Params {
-    int rows_valid, d, accumulate;
-    float* dW;
+    CUtensorMap tm;        // dW [V][d] fp32, box {32, 128}, 128-byte swizzle
+    int accumulate;
   };
   __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr) {
-    const bool valid = r < P.rows_valid;
-    float* out = P.dW + (size_t)r * P.d;
+  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr, EpiCtx& cx) {
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       float v[32];
       __syncwarp();
       tmem_ld_32x32b_x32(taddr + j * 32, v);
-      const int c0 = n * BN + j * 32;
-      if (valid) {
+      uint32_t w[32];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (c0 + 4 * t + 4 <= P.d) {
-            float4* p = reinterpret_cast<float4*>(out + c0 + 4 * t);
-            float4 w = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
-            if (P.accumulate) {
-              const float4 o = *p;
-              w.x += o.x; w.y += o.y; w.z += o.z; w.w += o.w;
-            }
-            *p = w;
-          }
-        }
-      }
+      for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+      stage_store(cx, &P.tm, n * BN + j * 32, cx.row_base, w, P.accumulate != 0);
     }
   }
 };

@@ -91,17 +91,19 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// Row-major bf16 matrix [outer][inner] with row pitch `pitch` elements,
-// 128-byte-swizzled boxes of box_inner x box_outer, zero fill out of bounds.
+// Row-major matrix [outer][inner] (bf16, or fp32 when `f32`) with row pitch
+// `pitch` elements, 128-byte-swizzled boxes of box_inner x box_outer; loads
+// out of bounds read zeros, stores out of bounds are dropped.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, bool f32 = false) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {pitch * 2};
+  cuuint64_t strides[1] = {pitch * (f32 ? 4 : 2)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -325,9 +327,10 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, nullptr, 0, 1, grad_loss, cscale);
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
 
-  CUtensorMap tmHk, tmWk, tmWmn, tmHmn;
+  CUtensorMap tmHk, tmWk, tmWmn, tmHmn, tmDW;
   if (!make_map(&tmHk, H, d, N, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, GeoP::B_ROWS) ||
-      !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, H, d, N, d, 64, BK))
+      !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, H, d, N, d, 64, BK) ||
+      !make_map(&tmDW, dW, d, V, d, 32, BM, true))
     return KD_ERR_CUDA;
   const int groups = resident_groups(dev);
 
@@ -354,7 +357,7 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     e3.lse = lse;
     e3.mask = mask;
     e3.cscale = cscale;
-    e3.dz = dz;
+    e3.tm = tmZk;
     if (launch_gemm<EpiDz, false, false, kPair>(1, dev, grid_for(a3.raster, groups), tmHk, tmWk, a3, e3, s) != cudaSuccess)
       return KD_ERR_CUDA;
 
@@ -364,10 +367,7 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     a4.num_kb = (int)ceil_div(V, BK);
     a4.status = status;
     EpiDh::Params e4{};
-    e4.rows_valid = (int)Cc;
-    e4.row0 = (int)c0;
-    e4.d = (int)d;
-    e4.dH = static_cast<__nv_bfloat16*>(dH);
+    if (!make_map(&e4.tm, static_cast<__nv_bfloat16*>(dH) + c0 * d, d, Cc, d, 64, BM)) return KD_ERR_CUDA;
     if (launch_gemm<EpiDh, false, true, kPair>(2, dev, grid_for(a4.raster, groups), tmZk, tmWmn, a4, e4, s) != cudaSuccess)
       return KD_ERR_CUDA;
 
@@ -378,10 +378,8 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     a5.b_k0 = (int)c0;
     a5.status = status;
     EpiDw::Params e5{};
-    e5.rows_valid = (int)V;
-    e5.d = (int)d;
+    e5.tm = tmDW;
     e5.accumulate = (accumulate_dW || c0 > 0) ? 1 : 0;
-    e5.dW = dW;
     if (launch_gemm<EpiDw, true, true, kPair>(3, dev, grid_for(a5.raster, groups), tmZmn, tmHmn, a5, e5, s) != cudaSuccess)
       return KD_ERR_CUDA;
   }
