@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 DEFAULT_CONFIG = 3
 L2_BYTES = 126 * 2**20
 KERNEL_SOURCES = ["kd_gemm.cuh", "kd_ptx.cuh", "kd_schedule.h", "kd_small_kernels.cuh", "kd_topk_kl.cu"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_fwd_traffic.txt")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dominant_kernel_traffic.txt")
 
 
 # ---------------------------------------------------------------- helpers
@@ -64,9 +64,9 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload: str):
-    """DRAM bytes per launch of the forward GEMM from the committed ncu
-    summary, if it was taken on this workload and on the current sources."""
+def committed_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on this workload, for this kernel and on the current sources."""
     try:
         kv = {}
         with open(TRAFFIC_FILE) as f:
@@ -74,7 +74,8 @@ def committed_traffic(workload: str):
                 if ":" in line and not line.startswith("#"):
                     k, v = line.split(":", 1)
                     kv[k.strip()] = v.strip()
-        if kv.get("source_hash") != kernel_source_hash() or kv.get("workload") != workload:
+        if (kv.get("source_hash") != kernel_source_hash() or kv.get("workload") != workload
+                or kv.get("kernel") != kernel):
             return None
         return float(kv["dram_bytes_per_launch"])
     except Exception:
@@ -163,10 +164,41 @@ def barrier(world: int):
 def launches_per_step(N: int, chunk: int) -> int:
     """Kernels this library launches for one forward + one backward call:
     forward = teacher prep, logits/lse GEMM, lse merge, finalize;
-    backward = teacher prep, finalize, and per chunk dZ, dH and dW GEMMs."""
+    backward = teacher prep, gradient scale, and per chunk the dZ recompute
+    GEMM and the joint dH/dW GEMM."""
     if N == 0:
         return 0
-    return 4 + 2 + 3 * math.ceil(N / chunk)
+    return 4 + 2 + 2 * math.ceil(N / chunk)
+
+
+def per_kernel_times(ev_b, ev_f, N, d, V, chunk):
+    """Live per-kernel totals from the events recorded around every backward
+    launch (launch 0 teacher prep, 1 gradient scale, then per chunk c the
+    dZ recompute 2+2c and the joint dH/dW GEMM 3+2c) and around the forward
+    call (its GEMM plus three sub-0.2 ms kernels)."""
+    steps = len(ev_b)
+    out = {"forward_gemm": {"launches": steps, "ms": sum(a.elapsed_time(b) for a, b in ev_f),
+                            "flops": 2.0 * N * d * V * steps}}
+    names = {0: "teacher_prep", 1: "grad_scale"}
+    for row in ev_b:
+        for j in range(len(row) - 1):
+            if j in names:
+                key, flops = names[j], 0.0
+            else:
+                c = (j - 2) // 2
+                cc = min(chunk, N - c * chunk)
+                key, flops = (("dz_recompute", 2.0 * cc * d * V) if j % 2 == 0
+                              else ("grads_dH_dW", 4.0 * cc * d * V))
+            k = out.setdefault(key, {"launches": 0, "ms": 0.0, "flops": 0.0})
+            k["launches"] += 1
+            k["ms"] += row[j].elapsed_time(row[j + 1])
+            k["flops"] += flops
+    total = sum(k["ms"] for k in out.values())
+    for k in out.values():
+        k["avg_ms"] = k["ms"] / k["launches"]
+        k["share"] = k["ms"] / total if total > 0 else None
+        k["tflops"] = k["flops"] / (k["ms"] / 1e3) / 1e12 if k["flops"] > 0 else None
+    return out
 
 
 def blas_threads() -> int:
@@ -262,9 +294,15 @@ def run_cuda(args, cfg, world, rank, local):
     peak_gib = (torch.cuda.max_memory_allocated(dev) - base_mem) / 2**30
     ws_gib = ws.numel() / 2**30
 
-    # ---- kernel-only timed region (inputs resident in HBM)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # ---- kernel-only timed region (inputs resident in HBM).  The backward
+    # pass records an event around each of its kernel launches (same kernels
+    # and work as the plain call), which gives live per-kernel durations.
+    nl = kd.backward_launches(N, chunk)
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    ev_b = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(args.steps)]
+    for e in [x for pair in ev_f for x in pair] + [x for row in ev_b for x in row]:
+        e.record(stream)                     # creates the CUDA event behind each object
     sampler = ClockSampler(local) if not args.no_clocks else None
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -275,19 +313,19 @@ def run_cuda(args, cfg, world, rank, local):
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        ev[i][0].record(stream)
+        ev_f[i][0].record(stream)
         loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, workspace=ws)
-        ev[i][1].record(stream)
+        ev_f[i][1].record(stream)
         kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, lse,
-                    workspace=ws, dH=dH, dW=dW)
-        ev[i][2].record(stream)
+                    workspace=ws, dH=dH, dW=dW, events=ev_b[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     clocks = sampler.stop() if sampler else None
     ms_local = start.elapsed_time(end)
-    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    fwd_ms = [a.elapsed_time(b) for a, b in ev_f]
+    bwd_ms = [row[0].elapsed_time(row[-1]) for row in ev_b]
+    kern = per_kernel_times(ev_b, ev_f, N, d, V, chunk)
     ms = reduce_max(ms_local, world, dev)
     st, _ = kd.check(ws)
     if st != 0:
@@ -329,11 +367,10 @@ def run_cuda(args, cfg, world, rank, local):
     ms_step = ms / args.steps
     flops_step = 8.0 * N * d * V
     tflops = flops_step * world / (ms_step / 1e3) / 1e12
-    # Roofline of the single longest launch: the forward GEMM (logits + online
-    # lse + teacher gather).  Its call also holds three tiny CUDA-core kernels
-    # (teacher prep, lse merge, finalize), which are counted in its time.
+    # Roofline of the dominant kernel (largest share of the step's kernel time).
+    dom_name, dom = max(((k, v) for k, v in kern.items() if v["flops"] > 0), key=lambda kv: kv[1]["ms"])
+    dom_ach = dom["tflops"]
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
-    fwd_ach = 2.0 * N * d * V / (fwd_avg / 1e3) / 1e12
     bwd_avg = sum(bwd_ms) / len(bwd_ms)
     peak_sus = peaks["bf16_tflops_sustained"]
     cpu = None
@@ -355,12 +392,14 @@ def run_cuda(args, cfg, world, rank, local):
         "config": config_block(cfg, world),
         "clocks": clocks,
         "gpu_launches": launches_per_step(N, chunk) * args.steps,
-        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel<EpiFwd> (forward logits/lse/gather)",
-                     "achieved": fwd_ach, "peak": peak_sus, "unit": "TFLOP/s", "frac": fwd_ach / peak_sus,
+        "roofline": {"bound": "tensor", "kernel": dom_name,
+                     "achieved": dom_ach, "peak": peak_sus, "unit": "TFLOP/s", "frac": dom_ach / peak_sus,
                      "peak_kind": f"bf16_tflops_sustained ({peaks_src})",
-                     "frac_of_burst": fwd_ach / peaks["bf16_tflops"],
-                     "flops_per_launch": 2.0 * N * d * V,
-                     "traffic": committed_traffic(cfg.name)},
+                     "frac_of_burst": dom_ach / peaks["bf16_tflops"],
+                     "flops_per_launch": dom["flops"] / dom["launches"],
+                     "avg_launch_ms": dom["avg_ms"], "share": dom["share"],
+                     "traffic": committed_traffic(cfg.name, dom_name)},
+        "kernels": {k: {kk: v[kk] for kk in ("launches", "avg_ms", "share", "tflops")} for k, v in kern.items()},
         "roofline_step": {"bound": "tensor", "achieved": tflops / world, "peak": peak_sus,
                           "unit": "TFLOP/s", "frac": tflops / world / peak_sus,
                           "flops_per_step": flops_step},

@@ -27,6 +27,7 @@ EXPORTS = (
     "kd_topk_kl_backward",
     "kd_topk_kl_check",
     "kd_topk_kl_forward_noalloc",
+    "kd_topk_kl_backward_profiled",
 )
 
 _lib = None
@@ -52,6 +53,9 @@ def load() -> ctypes.CDLL:
         lib.kd_topk_kl_backward.restype = i32
         lib.kd_topk_kl_check.argtypes = [p, p, ctypes.POINTER(i64)]
         lib.kd_topk_kl_check.restype = i32
+        lib.kd_topk_kl_backward_profiled.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p,
+                                                     p, i32, p, sz, p, ctypes.POINTER(ctypes.c_void_p), i64]
+        lib.kd_topk_kl_backward_profiled.restype = i32
         lib.kd_topk_kl_forward_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, p, p, p]
         lib.kd_topk_kl_forward_noalloc.restype = i32
         _lib = lib
@@ -83,6 +87,17 @@ def kd_topk_kl_backward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, 
     return int(load().kd_topk_kl_backward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk,
                                           lse, grad_loss, dH, dW, int(accumulate_dW), workspace,
                                           workspace_bytes, stream))
+
+
+def kd_topk_kl_backward_profiled(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse,
+                                 grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes, stream,
+                                 events) -> int:
+    """``events``: a sequence of cudaEvent_t handles (ints), one more than
+    the backward pass's launches (2 + 2 * ceil(N / chunk))."""
+    arr = (ctypes.c_void_p * len(events))(*events)
+    return int(load().kd_topk_kl_backward_profiled(H, W, topk_idx, topk_logit, mask, N, d, V, K, T,
+                                                   chunk, lse, grad_loss, dH, dW, int(accumulate_dW),
+                                                   workspace, workspace_bytes, stream, arr, len(events)))
 
 
 def kd_topk_kl_check(workspace, stream) -> tuple[int, int]:

@@ -70,11 +70,18 @@ def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 
     return loss, lse
 
 
+def backward_launches(N: int, chunk: int) -> int:
+    """Kernel launches of one backward call (see kd_topk_kl_backward_profiled)."""
+    return 0 if N == 0 else 2 + 2 * ((N + chunk - 1) // chunk)
+
+
 def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.Tensor,
              grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
              accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
-             dH: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Returns (dH [N,d] bf16, dW [V,d] fp32)."""
+             dH: Optional[torch.Tensor] = None, events=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Returns (dH [N,d] bf16, dW [V,d] fp32).  With ``events`` (a list of
+    backward_launches(N, chunk) + 1 created torch.cuda.Event objects) the
+    library records them around each of its kernel launches."""
     N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
     dev = H.device
     if workspace is None:
@@ -87,11 +94,18 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
     if grad_loss is not None:
         grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
-                                  N, d, V, K, float(T), int(chunk), _ptr(lse), _ptr(grad_loss),
-                                  _ptr(dH), _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
-                                  workspace.numel(), stream)
-    _raise(st, "kd_topk_kl_backward")
+    if events is None:
+        st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                      N, d, V, K, float(T), int(chunk), _ptr(lse), _ptr(grad_loss),
+                                      _ptr(dH), _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
+                                      workspace.numel(), stream)
+        _raise(st, "kd_topk_kl_backward")
+    else:
+        st = _abi.kd_topk_kl_backward_profiled(
+            _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
+            int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+            _ptr(workspace), workspace.numel(), stream, [e.cuda_event for e in events])
+        _raise(st, "kd_topk_kl_backward_profiled")
     return dH, dW
 
 

@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "kd_ptx.cuh"
 #include "kd_schedule.h"
 #include "kd_small_kernels.cuh"
@@ -37,25 +39,54 @@ constexpr int TMEM_COLS = 512;
 // computes a 256 x 256 tile with cta_group::2 MMAs; each CTA stages its own
 // 128 rows of A and 128 rows of B, holds its 128 accumulator rows in its own
 // tensor memory, and the pair leader issues the MMAs.
-template <bool PAIR>
+template <bool PAIR, bool STAGING = true>
 struct Geo {
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;          // B rows staged per CTA
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // per CTA
-  static constexpr int STAGES = PAIR ? 6 : 4;
-  static constexpr int STAGING_BYTES = 2 * BM * 128;           // two 128-row x 128-byte store buffers
+  // Epilogues that store through shared memory need two 16 KB staging
+  // buffers; without them the pair variant fits a seventh stage.
+  static constexpr int STAGES = PAIR ? (STAGING ? 6 : 7) : 4;
+  static constexpr int STAGING_BYTES = STAGING ? 2 * BM * 128 : 0;  // two 128-row x 128-byte buffers
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // per stage, whole tile
 };
 
-struct GemmArgs {
+constexpr int kMaxGroups = 160;   // >= resident CTAs (or CTA pairs) on one GPU
+
+// One GEMM as the kernel sees it: its tile schedule, K blocks per tile, and
+// offsets added to the tensor-map coordinates of A and B.
+struct ProbArgs {
   Raster raster;
   int num_kb;           // BK-wide K blocks per tile
-  int a_row0, b_row0;   // tensor-map offsets added to the row (M / N) coordinate
-  int a_k0, b_k0;       // tensor-map offsets added to the K coordinate
+  int a_row0, b_row0;   // added to the row (M / N) coordinate
+  int a_k0, b_k0;       // added to the K coordinate
+};
+
+// A launch runs problem 0 and, optionally, problem 1.  Problem 0's units go
+// round-robin over the groups (CTAs, or CTA pairs); problem 1's units are
+// split into one contiguous range per group, [p1_start[g], p1_start[g+1]),
+// sized on the host so that every group gets about the same number of K
+// blocks in total.  Every role of a group walks the same sequence.
+struct GemmArgs {
+  ProbArgs prob[2];
+  int p1_start[kMaxGroups + 1];
   Status* status;
+};
+
+// Compile-time description of a problem: its epilogue and operand majorness.
+template <class EpiT, bool AMN, bool BMN>
+struct Prob {
+  using Epi = EpiT;
+  static constexpr bool A_MN = AMN, B_MN = BMN, present = true;
+};
+
+struct EpiNone;
+struct NoProb {
+  using Epi = EpiNone;
+  static constexpr bool A_MN = false, B_MN = false, present = false;
 };
 
 // Loads one operand tile (rows x BK) for K block kb into shared memory.
@@ -125,189 +156,277 @@ __device__ __forceinline__ void stage_store(EpiCtx& cx, const CUtensorMap* tm, i
   ++cx.seq;
 }
 
-template <class Epi, bool A_MN, bool B_MN, bool PAIR>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const GemmArgs args, const __grid_constant__ typename Epi::Params ep) {
-  using G = Geo<PAIR>;
-  constexpr int STAGES = G::STAGES;
-  extern __shared__ uint8_t smem_raw[];
+template <bool FIRST, class A, class B>
+__device__ __forceinline__ auto& pick(A& a, B& b) {
+  if constexpr (FIRST) return a; else return b;
+}
+
+// ---------------------------------------------------------------- pipeline roles
+//
+// Shared-memory layout of a GEMM CTA (G = Geo<...>): STAGES operand stages,
+// the epilogue's staging buffers, then the mbarriers:
+//   full[s]   stage s loaded (TMA bytes of both CTAs of a pair, on the leader)
+//   empty[s]  stage s consumed by the MMAs (commit, multicast to the pair)
+//   tfull[a]  accumulator a written (commit, multicast to the pair)
+//   tempty[a] accumulator a drained by every epilogue thread (on the leader)
+// followed by the tensor-memory address slot and the CTA's abort flag.
+template <class G>
+struct Smem {
+  uint32_t sbase, staging, bar_base;
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  __device__ __forceinline__ uint32_t full(int s) const { return bar_base + 8u * s; }
+  __device__ __forceinline__ uint32_t empty(int s) const { return bar_base + 8u * (G::STAGES + s); }
+  __device__ __forceinline__ uint32_t tfull(int a) const { return bar_base + 8u * (2 * G::STAGES + a); }
+  __device__ __forceinline__ uint32_t tempty(int a) const { return bar_base + 8u * (2 * G::STAGES + 2 + a); }
+};
+
+template <class G>
+__device__ __forceinline__ Smem<G> smem_layout(uint8_t* smem_raw) {
+  Smem<G> L;
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t staging = sbase + STAGES * G::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * G::STAGE_BYTES + G::STAGING_BYTES);
-  const uint32_t bar_base = smem_u32(bars);
-  auto full_bar = [&](int s) { return bar_base + 8u * s; };
-  auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
-  auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + a); };
-  auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  L.sbase = smem_u32(smem);
+  L.staging = L.sbase + G::STAGES * G::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES + G::STAGING_BYTES);
+  L.bar_base = smem_u32(bars);
+  L.tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * G::STAGES + 4);
+  L.abort_flag = reinterpret_cast<volatile int*>(L.tmem_slot + 1);
+  return L;
+}
 
+// Barrier init and tensor-memory allocation; returns the TMEM base address.
+template <class G, bool PAIR>
+__device__ __forceinline__ uint32_t pipeline_setup(const Smem<G>& L) {
   const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const Raster& R = args.raster;
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;       // CTA within the pair
-  const int group = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int ngroups = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  // Barriers that the pair leader owns: stage-full (TMA bytes of both CTAs)
-  // and accumulator-empty (epilogue threads of both CTAs).
-  auto leader = [&](uint32_t a) { return PAIR ? mapa_shared(a, 0) : a; };
-
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < G::STAGES; ++s) {
+      mbar_init(L.full(s), 1);
+      mbar_init(L.empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), (PAIR ? 2 : 1) * 4 * 32);
+      mbar_init(L.tfull(a), 1);
+      mbar_init(L.tempty(a), (PAIR ? 2 : 1) * 4 * 32);
     }
-    *abort_flag = 0;
+    *L.abort_flag = 0;
     fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
     if constexpr (PAIR) {
-      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_alloc_pair(smem_u32(L.tmem_slot), TMEM_COLS);
       tmem_relinquish_pair();
     } else {
-      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_alloc(smem_u32(L.tmem_slot), TMEM_COLS);
       tmem_relinquish();
     }
   }
   tc_fence_before();
   if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
+  return *L.tmem_slot;
+}
 
-  bool failed = false;
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (every CTA)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int u = group; u < R.num_units && !failed; u += ngroups) {
-        int m, split, n0, n1;
-        decode_unit(R, u, m, split, n0, n1);
-        for (int n = n0; n < n1 && !failed; ++n) {
-          for (int kb = 0; kb < args.num_kb; ++kb) {
-            if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag)) { failed = true; break; }
-            const uint32_t sa = sbase + stage * G::STAGE_BYTES;
-            const uint32_t sb = sa + G::A_BYTES;
-            const uint32_t fb = leader(full_bar(stage));
-            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), G::TX_BYTES);
-            load_operand<A_MN, BM, PAIR>(sa, &tmA, args.a_row0 + m * G::TILE_M + (int)rank * BM,
-                                         args.a_k0 + kb * BK, fb);
-            load_operand<B_MN, G::B_ROWS, PAIR>(sb, &tmB, args.b_row0 + n * BN + (int)rank * G::B_ROWS,
-                                                args.b_k0 + kb * BK, fb);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (pair leader)
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(G::TILE_M, BN, A_MN, B_MN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      for (int u = group; u < R.num_units && !failed; u += ngroups) {
-        int m, split, n0, n1;
-        decode_unit(R, u, m, split, n0, n1);
-        for (int n = n0; n < n1 && !failed; ++n) {
-          if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { failed = true; break; }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + acc * BN;
-          for (int kb = 0; kb < args.num_kb; ++kb) {
-            if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag)) { failed = true; break; }
-            tc_fence_after();
-            const uint32_t sa = sbase + stage * G::STAGE_BYTES;
-            const uint32_t sb = sa + G::A_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-              const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-              if constexpr (PAIR)
-                tc_mma_bf16_pair(d_tmem, operand_desc<A_MN>(sa, kk), operand_desc<B_MN>(sb, kk), idesc, accum);
-              else
-                tc_mma_bf16(d_tmem, operand_desc<A_MN>(sa, kk), operand_desc<B_MN>(sb, kk), idesc, accum);
-            }
-            if constexpr (PAIR) tc_commit_pair_mc(empty_bar(stage), 0x3); else tc_commit(empty_bar(stage));
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          }
-          if (failed) break;
-          if constexpr (PAIR) tc_commit_pair_mc(tfull_bar(acc), 0x3); else tc_commit(tfull_bar(acc));
-          acc ^= 1;
-          if (acc == 0) acc_phase ^= 1u;
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue (every CTA)
-    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int row = (int)rank * BM + q * 32 + lane;   // row of the tile owned by this thread
-    const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    Epi epi;
-    EpiCtx cx;
-    cx.stage[0] = staging;
-    cx.stage[1] = staging + BM * 128;
-    cx.rr = q * 32 + lane;
-    cx.issuer = (threadIdx.x == 64);
-    cx.seq = 0;
-    for (int u = group; u < R.num_units && !failed; u += ngroups) {
-      int m, split, n0, n1;
-      decode_unit(R, u, m, split, n0, n1);
-      const int grow = m * G::TILE_M + row;
-      cx.row_base = m * G::TILE_M + (int)rank * BM;
-      epi.begin_unit(ep, grow, split, n0);
-      for (int n = n0; n < n1; ++n) {
-        // One outcome for all 128 epilogue threads: tcgen05.ld needs whole
-        // warps and the store path synchronises the four warps.
-        const bool ok = epilogue_bar_and(128, mbar_wait_bounded(tfull_bar(acc), acc_phase, abort_flag));
-        if (!ok) { failed = true; break; }
-        tc_fence_after();
-        epi.tile(ep, grow, n, lane_addr + acc * BN, cx);
-        tc_fence_before();
-        if constexpr (PAIR) mbar_arrive_cluster(leader(tempty_bar(acc)));
-        else mbar_arrive(tempty_bar(acc));
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-      }
-      if (failed) break;
-      epi.end_unit(ep, grow, split);
-    }
-    if (cx.issuer) bulk_wait<0>();          // every TMA store of this CTA has completed
-  }
-
+// Records a failure, lets issued asynchronous work land, and releases the
+// tensor memory once neither CTA of a pair can still touch the other's.
+template <class G, bool PAIR>
+__device__ __forceinline__ void pipeline_teardown(const Smem<G>& L, bool failed, Status* status,
+                                                  uint32_t tmem_base) {
   if (failed) {
-    *abort_flag = 1;
-    atomicOr(&args.status->timeout, 1u);
+    *L.abort_flag = 1;
+    atomicOr(&status->timeout, 1u);
   }
   __syncwarp();
   __syncthreads();
-  if (*abort_flag) {
-    // Let asynchronous copies and MMAs that were already issued land before
-    // the CTA releases its shared and tensor memory.
+  if (*L.abort_flag) {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 2000000ull) { }
     __syncthreads();
   }
-  // Neither CTA of a pair may release its memory while the leader's MMAs can
-  // still read the peer's shared memory or write its tensor memory.
   if constexpr (PAIR) cluster_sync_all();
-  if (warp == 1) {
+  if ((threadIdx.x >> 5) == 1) {
     tc_fence_after();
     if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
     else tmem_dealloc(tmem_base, TMEM_COLS);
   }
+}
+
+// Per-role pipeline position, carried across units and problems.
+struct RoleState {
+  int stage = 0;
+  uint32_t phase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+};
+
+// TMA producer: all K blocks of every tile of unit u.
+template <class G, bool PAIR, class P>
+__device__ __forceinline__ bool produce_unit(const Smem<G>& L, RoleState& st, uint32_t rank,
+                                             const ProbArgs& pa, const CUtensorMap* tA,
+                                             const CUtensorMap* tB, int u) {
+  int m, split, n0, n1;
+  decode_unit(pa.raster, u, m, split, n0, n1);
+  for (int n = n0; n < n1; ++n) {
+    for (int kb = 0; kb < pa.num_kb; ++kb) {
+      if (!mbar_wait_bounded(L.empty(st.stage), st.phase ^ 1u, L.abort_flag)) return false;
+      const uint32_t sa = L.sbase + st.stage * G::STAGE_BYTES;
+      const uint32_t sb = sa + G::A_BYTES;
+      const uint32_t fb = PAIR ? mapa_shared(L.full(st.stage), 0) : L.full(st.stage);
+      if (rank == 0) mbar_arrive_expect_tx(L.full(st.stage), G::TX_BYTES);
+      load_operand<P::A_MN, BM, PAIR>(sa, tA, pa.a_row0 + m * G::TILE_M + (int)rank * BM,
+                                      pa.a_k0 + kb * BK, fb);
+      load_operand<P::B_MN, G::B_ROWS, PAIR>(sb, tB, pa.b_row0 + n * BN + (int)rank * G::B_ROWS,
+                                             pa.b_k0 + kb * BK, fb);
+      if (++st.stage == G::STAGES) { st.stage = 0; st.phase ^= 1u; }
+    }
+  }
+  return true;
+}
+
+// MMA issuer (pair leader, one thread): every tile of unit u into the next
+// free accumulator.
+template <class G, bool PAIR, class P>
+__device__ __forceinline__ bool mma_unit(const Smem<G>& L, RoleState& st, uint32_t tmem_base,
+                                         const ProbArgs& pa, int u) {
+  constexpr uint32_t idesc = idesc_bf16_f32(G::TILE_M, BN, P::A_MN, P::B_MN);
+  int m, split, n0, n1;
+  decode_unit(pa.raster, u, m, split, n0, n1);
+  for (int n = n0; n < n1; ++n) {
+    if (!mbar_wait_bounded(L.tempty(st.acc), st.acc_phase ^ 1u, L.abort_flag)) return false;
+    tc_fence_after();
+    const uint32_t d_tmem = tmem_base + st.acc * BN;
+    for (int kb = 0; kb < pa.num_kb; ++kb) {
+      if (!mbar_wait_bounded(L.full(st.stage), st.phase, L.abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sa = L.sbase + st.stage * G::STAGE_BYTES;
+      const uint32_t sb = sa + G::A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+        const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+        if constexpr (PAIR)
+          tc_mma_bf16_pair(d_tmem, operand_desc<P::A_MN>(sa, kk), operand_desc<P::B_MN>(sb, kk), idesc, accum);
+        else
+          tc_mma_bf16(d_tmem, operand_desc<P::A_MN>(sa, kk), operand_desc<P::B_MN>(sb, kk), idesc, accum);
+      }
+      if constexpr (PAIR) tc_commit_pair_mc(L.empty(st.stage), 0x3); else tc_commit(L.empty(st.stage));
+      if (++st.stage == G::STAGES) { st.stage = 0; st.phase ^= 1u; }
+    }
+    if constexpr (PAIR) tc_commit_pair_mc(L.tfull(st.acc), 0x3); else tc_commit(L.tfull(st.acc));
+    st.acc ^= 1;
+    if (st.acc == 0) st.acc_phase ^= 1u;
+  }
+  return true;
+}
+
+// Epilogue (all 128 threads of warps 2-5): drain each tile of unit u.
+template <class G, bool PAIR, class Epi>
+__device__ __forceinline__ bool epi_unit(const Smem<G>& L, RoleState& st, uint32_t rank,
+                                         uint32_t lane_addr, int row, Epi& epi,
+                                         const typename Epi::Params& ep, const CUtensorMap* out,
+                                         const ProbArgs& pa, int u, EpiCtx& cx) {
+  int m, split, n0, n1;
+  decode_unit(pa.raster, u, m, split, n0, n1);
+  const int grow = m * G::TILE_M + row;
+  cx.row_base = m * G::TILE_M + (int)rank * BM;
+  epi.begin_unit(ep, grow, split, n0);
+  for (int n = n0; n < n1; ++n) {
+    // One outcome for all 128 epilogue threads: tcgen05.ld needs whole
+    // warps and the store path synchronises the four warps.
+    const bool ok = epilogue_bar_and(128, mbar_wait_bounded(L.tfull(st.acc), st.acc_phase, L.abort_flag));
+    if (!ok) return false;
+    tc_fence_after();
+    epi.tile(ep, out, grow, n, lane_addr + st.acc * BN, cx);
+    tc_fence_before();
+    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(L.tempty(st.acc), 0));
+    else mbar_arrive(L.tempty(st.acc));
+    st.acc ^= 1;
+    if (st.acc == 0) st.acc_phase ^= 1u;
+  }
+  epi.end_unit(ep, grow, split);
+  return true;
+}
+
+__device__ __forceinline__ EpiCtx make_epi_ctx(uint32_t staging) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  EpiCtx cx;
+  cx.stage[0] = staging;
+  cx.stage[1] = staging + BM * 128;
+  cx.rr = (warp & 3) * 32 + lane;
+  cx.issuer = (threadIdx.x == 64);
+  cx.seq = 0;
+  cx.row_base = 0;
+  return cx;
+}
+
+// One or two GEMM problems per launch (see GemmArgs).  tmO0 / tmO1 are the
+// output maps of epilogues that store through TMA (unused otherwise).
+template <class P0, class P1, bool PAIR>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+               const __grid_constant__ CUtensorMap tmO0,
+               const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+               const __grid_constant__ CUtensorMap tmO1,
+               const __grid_constant__ GemmArgs args,
+               const __grid_constant__ typename P0::Epi::Params ep0,
+               const __grid_constant__ typename P1::Epi::Params ep1) {
+  using G = Geo<PAIR, P0::Epi::kStaging || P1::Epi::kStaging>;
+  extern __shared__ uint8_t smem_raw[];
+  const Smem<G> L = smem_layout<G>(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int group = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int ngroups = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    if constexpr (P1::present) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
+  }
+  const uint32_t tmem_base = pipeline_setup<G, PAIR>(L);
+
+  // This group's units: problem 0 round-robin, then problem 1's range.
+  auto for_each_unit = [&](auto&& body) {
+    bool ok = true;
+    for (int u = group; ok && u < args.prob[0].raster.num_units; u += ngroups)
+      ok = body(P0{}, args.prob[0], &tmA0, &tmB0, u);
+    if constexpr (P1::present) {
+      for (int u = args.p1_start[group]; ok && u < args.p1_start[group + 1]; ++u)
+        ok = body(P1{}, args.prob[1], &tmA1, &tmB1, u);
+    }
+    return ok;
+  };
+
+  bool failed = false;
+  RoleState st;
+  if (warp == 0) {
+    if (lane == 0)
+      failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap* tA,
+                                  const CUtensorMap* tB, int u) {
+        return produce_unit<G, PAIR, decltype(pt)>(L, st, rank, pa, tA, tB, u);
+      });
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0)
+      failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap*, const CUtensorMap*,
+                                  int u) { return mma_unit<G, PAIR, decltype(pt)>(L, st, tmem_base, pa, u); });
+  } else {
+    const int q = warp & 3;
+    const int row = (int)rank * BM + q * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(q * 32) << 16);
+    typename P0::Epi epi0;
+    typename P1::Epi epi1;
+    EpiCtx cx = make_epi_ctx(L.staging);
+    failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap*, const CUtensorMap*,
+                                int u) {
+      using P = decltype(pt);
+      constexpr bool first = std::is_same<P, P0>::value;
+      return epi_unit<G, PAIR>(L, st, rank, lane_addr, row, pick<first>(epi0, epi1), pick<first>(ep0, ep1),
+                               first ? &tmO0 : &tmO1, pa, u, cx);
+    });
+    if (cx.issuer) bulk_wait<0>();          // every TMA store of this CTA has completed
+  }
+  pipeline_teardown<G, PAIR>(L, failed, args.status, tmem_base);
 }
 
 // ---------------------------------------------------------------- epilogues
@@ -325,6 +444,7 @@ __device__ __forceinline__ int lower_bound_row(const int32_t* row, int len, int 
 // gathered sum of p * z at the teacher's columns; one (m, s, g) partial per
 // token per split.  Columns >= V are -inf.
 struct EpiFwd {
+  static constexpr bool kStaging = false;
   struct Params {
     int N, V, Kp;
     const int32_t* tidx;
@@ -354,7 +474,8 @@ struct EpiFwd {
     }
   }
 
-  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr, EpiCtx&) {
+  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap*, int, int n, uint32_t taddr,
+                                       EpiCtx&) {
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       float v[32];
@@ -406,11 +527,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // Backward, per chunk: dZ = c_n (exp(z - lse_n) - p at the teacher's columns),
-// rounded to bf16 and stored for the chunk's tokens (row-major, ldz columns;
-// columns in [V, ldz) are written as 0) through shared memory and TMA.
+// rounded to bf16 and stored for the chunk's tokens (row-major, ldz columns)
+// through shared memory and TMA (`out`: the chunk buffer, bf16, box
+// {64, 128}, 128-byte swizzle).  Columns in [V, ldz) and rows at or past the
+// chunk's end (up to the buffer's rows) are written as 0, so that a buffer
+// reused for a shorter last chunk holds no stale rows.
 struct EpiDz {
+  static constexpr bool kStaging = true;
   struct Params {
-    CUtensorMap tm;        // dZ chunk [rows_valid][ldz] bf16, box {64, 128}, 128-byte swizzle
     int rows_valid;        // tokens in this chunk
     int row0;              // global token index of chunk row 0
     int V, ldz, Kp;
@@ -423,7 +547,8 @@ struct EpiDz {
   __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int r, int n, uint32_t taddr, EpiCtx& cx) {
+  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int r, int n,
+                                       uint32_t taddr, EpiCtx& cx) {
     const bool valid = r < P.rows_valid;
     const int grow = P.row0 + r;
     float L = 0.f, c = 0.f;
@@ -465,25 +590,28 @@ struct EpiDz {
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float a = (c0 + 2 * i < P.V) ? c * v[2 * i] : 0.f;
-        const float b = (c0 + 2 * i + 1 < P.V) ? c * v[2 * i + 1] : 0.f;
+        const float a = (valid && c0 + 2 * i < P.V) ? c * v[2 * i] : 0.f;
+        const float b = (valid && c0 + 2 * i + 1 < P.V) ? c * v[2 * i + 1] : 0.f;
         w[i] = pack_bf16x2(a, b);
       }
-      stage_store(cx, &P.tm, c0, cx.row_base, w, false);
+      stage_store(cx, out, c0, cx.row_base, w, false);
     }
   }
 };
 
 // Backward, per chunk: dH rows of the chunk's tokens, bf16, through shared
-// memory and TMA (the map covers the chunk's rows only).
+// memory and TMA (`out`: dH [N][d] bf16, box {64, 128}, 128-byte swizzle;
+// chunk row r is dH row row0 + r).
 struct EpiDh {
+  static constexpr bool kStaging = true;
   struct Params {
-    CUtensorMap tm;        // dH rows of the chunk [rows][d] bf16, box {64, 128}, 128-byte swizzle
+    int row0;
   };
   __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr, EpiCtx& cx) {
+  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int, int n,
+                                       uint32_t taddr, EpiCtx& cx) {
 #pragma unroll 1
     for (int j = 0; j < BN / 64; ++j) {
       float v[64];
@@ -495,7 +623,7 @@ struct EpiDh {
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-      stage_store(cx, &P.tm, n * BN + j * 64, cx.row_base, w, false);
+      stage_store(cx, out, n * BN + j * 64, P.row0 + cx.row_base, w, false);
     }
   }
 };
@@ -504,14 +632,15 @@ struct EpiDh {
 // per CTA, fp32, stored (first chunk without accumulation) or added in place
 // by TMA reductions: the memory system does the read-modify-write.
 struct EpiDw {
+  static constexpr bool kStaging = true;
   struct Params {
-    CUtensorMap tm;        // dW [V][d] fp32, box {32, 128}, 128-byte swizzle
-    int accumulate;
+    int accumulate;        // `out`: dW [V][d] fp32, box {32, 128}, 128-byte swizzle
   };
   __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
-  __device__ __forceinline__ void tile(const Params& P, int, int n, uint32_t taddr, EpiCtx& cx) {
+  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int, int n,
+                                       uint32_t taddr, EpiCtx& cx) {
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       float v[32];
@@ -520,9 +649,20 @@ struct EpiDw {
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
-      stage_store(cx, &P.tm, n * BN + j * 32, cx.row_base, w, P.accumulate != 0);
+      stage_store(cx, out, n * BN + j * 32, cx.row_base, w, P.accumulate != 0);
     }
   }
+};
+
+// Placeholder epilogue of an absent second problem.
+struct EpiNone {
+  static constexpr bool kStaging = false;
+  struct Params {
+    int unused;
+  };
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void tile(const Params&, const CUtensorMap*, int, int, uint32_t, EpiCtx&) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 };
 
 }  // namespace kd

@@ -45,7 +45,7 @@ KD_HD void decode_unit(const Raster& r, int u, int& m, int& split, int& n0, int&
 
 // One tile per unit; bands fastest (group_m = all bands) or column tiles
 // fastest (group_m = 1).
-inline Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
+KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
   Raster r;
   r.m_tiles = (int)m_tiles;
   r.n_tiles = (int)n_tiles;
@@ -78,6 +78,44 @@ inline Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid) {
   r.group_m = gm < 1 ? 1 : (gm > m_tiles ? (int)m_tiles : gm);
   r.num_units = (int)(m_tiles * r.splits);
   return r;
+}
+
+// Two problems in one launch: problem 0's U0 units (k0 K blocks each) go
+// round-robin over `groups`; problem 1's U1 units (k1 K blocks each) are cut
+// into one contiguous range per group, [starts[g], starts[g+1]), sized so
+// that every group's total K blocks are as equal as whole units allow
+// (largest remainders first).  starts has groups + 1 entries.
+inline void balance_ranges(int64_t U0, int64_t k0, int64_t U1, int64_t k1, int groups, int* starts) {
+  const double target = (double)(U0 * k0 + U1 * k1) / groups;
+  int64_t sum = 0;
+  int64_t cnt[256];
+  double frac[256];
+  for (int g = 0; g < groups; ++g) {
+    const int64_t n0 = g < U0 ? (U0 - g + groups - 1) / groups : 0;
+    double want = (target - (double)(n0 * k0)) / (double)(k1 > 0 ? k1 : 1);
+    if (want < 0) want = 0;
+    cnt[g] = (int64_t)want;
+    frac[g] = want - (double)cnt[g];
+    sum += cnt[g];
+  }
+  while (sum < U1) {
+    int best = 0;
+    for (int g = 1; g < groups; ++g)
+      if (frac[g] > frac[best]) best = g;
+    cnt[best] += 1;
+    frac[best] -= 1.0;
+    sum += 1;
+  }
+  while (sum > U1) {
+    int best = -1;
+    for (int g = 0; g < groups; ++g)
+      if (cnt[g] > 0 && (best < 0 || frac[g] < frac[best])) best = g;
+    cnt[best] -= 1;
+    frac[best] += 1.0;
+    sum -= 1;
+  }
+  starts[0] = 0;
+  for (int g = 0; g < groups; ++g) starts[g + 1] = starts[g] + (int)cnt[g];
 }
 
 }  // namespace kd

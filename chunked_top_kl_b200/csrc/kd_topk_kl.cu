@@ -60,7 +60,7 @@ Layout make_layout(int64_t N, int64_t V, int64_t K, int64_t chunk) {
   L.off_pm = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
-  L.off_dz = take(2 * (size_t)L.C * L.ldz);
+  L.off_dz = take(2 * (size_t)L.C * L.ldz);   // one dZ chunk (bf16)
   L.total = o;
   return L;
 }
@@ -132,18 +132,17 @@ int device_sms(int dev) {
 constexpr bool kPair = true;
 using GeoP = Geo<kPair>;
 
-template <class Epi, bool A_MN, bool B_MN, bool PAIR>
-cudaError_t launch_gemm(int slot, int dev, int groups, const CUtensorMap& ta, const CUtensorMap& tb,
-                        const GemmArgs& args, const typename Epi::Params& ep, cudaStream_t s) {
-  using G = Geo<PAIR>;
-  auto kern = gemm_tc_kernel<Epi, A_MN, B_MN, PAIR>;
+template <class P0, class P1, bool PAIR>
+cudaError_t launch_gemm(int slot, int dev, int groups, const CUtensorMap& ta0, const CUtensorMap& tb0,
+                        const CUtensorMap& to0, const CUtensorMap& ta1, const CUtensorMap& tb1,
+                        const CUtensorMap& to1, const GemmArgs& args,
+                        const typename P0::Epi::Params& ep0, const typename P1::Epi::Params& ep1,
+                        cudaStream_t s) {
+  using G = Geo<PAIR, P0::Epi::kStaging || P1::Epi::kStaging>;
+  auto kern = gemm_tc_kernel<P0, P1, PAIR>;
   if (dev >= 0 && dev < kMaxDevices && !g_dev[dev].attr_set[slot]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    if (PAIR) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-      (void)e;
-    }
     g_dev[dev].attr_set[slot] = true;
   }
   cudaLaunchConfig_t cfg = {};
@@ -158,9 +157,29 @@ cudaError_t launch_gemm(int slot, int dev, int groups, const CUtensorMap& ta, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args, ep);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta0, tb0, to0, ta1, tb1, to1, args, ep0, ep1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// One problem per launch.
+template <class P0>
+cudaError_t launch_one(int slot, int dev, int groups, const CUtensorMap& ta, const CUtensorMap& tb,
+                       const CUtensorMap& to, const ProbArgs& pa, Status* status,
+                       const typename P0::Epi::Params& ep, cudaStream_t s) {
+  GemmArgs a{};
+  a.prob[0] = pa;
+  a.status = status;
+  EpiNone::Params none{};
+  return launch_gemm<P0, NoProb, kPair>(slot, dev, groups, ta, tb, to, ta, tb, to, a, ep, none, s);
+}
+
+// Problem 0 round-robin, problem 1 in contiguous per-group ranges that even
+// out the groups' total K blocks (see balance_ranges).
+void balance_second_problem(GemmArgs& a, int groups) {
+  balance_ranges(a.prob[0].raster.num_units, (int64_t)a.prob[0].raster.tiles_per_split * a.prob[0].num_kb,
+                 a.prob[1].raster.num_units, (int64_t)a.prob[1].raster.tiles_per_split * a.prob[1].num_kb,
+                 groups, a.p1_start);
 }
 
 // Work groups (CTAs, or CTA pairs) that can be resident at once: one per SM,
@@ -170,12 +189,12 @@ int resident_groups(int dev) {
   if (!kPair) return sms;
   if (dev < 0 || dev >= kMaxDevices) return sms / 2;
   if (!g_dev[dev].pair_groups) {
-    auto kern = gemm_tc_kernel<EpiDz, false, false, true>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GeoP::SMEM_BYTES);
+    auto kern = gemm_tc_kernel<Prob<EpiDz, false, false>, NoProb, true>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<true, true>::SMEM_BYTES);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)sms, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = GeoP::SMEM_BYTES;
+    cfg.dynamicSmemBytes = Geo<true, true>::SMEM_BYTES;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -194,6 +213,11 @@ int resident_groups(int dev) {
 }
 
 inline int grid_for(const Raster& r, int groups) { return r.num_units < groups ? r.num_units : groups; }
+
+using ProbFwd = Prob<EpiFwd, false, false>;   // A = H (K-major), B = W (K-major)
+using ProbDz = Prob<EpiDz, false, false>;     // A = H chunk, B = W
+using ProbDh = Prob<EpiDh, false, true>;      // A = dZ (K-major over V), B = W (MN-major over d)
+using ProbDw = Prob<EpiDw, true, true>;       // A = dZ^T (MN-major over V), B = H chunk (MN-major over d)
 
 int common_checks(const void* H, const void* W, const int32_t* idx, const float* logit,
                   int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
@@ -268,10 +292,9 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   if (!make_map(&tmH, H, d, N, d, BK, BM) || !make_map(&tmW, W, d, V, d, BK, GeoP::B_ROWS))
     return KD_ERR_CUDA;
   const int groups = resident_groups(dev);
-  GemmArgs a{};
+  ProbArgs a{};
   a.raster = forward_raster(ceil_div(N, GeoP::TILE_M), ceil_div(V, BN), groups);
   a.num_kb = (int)ceil_div(d, BK);
-  a.status = status;
   EpiFwd::Params ep{};
   ep.N = (int)N;
   ep.V = (int)V;
@@ -281,7 +304,7 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   ep.part_m = at<float>(workspace, L.off_pm);
   ep.part_s = at<float>(workspace, L.off_ps);
   ep.part_g = at<float>(workspace, L.off_pg);
-  if (launch_gemm<EpiFwd, false, false, kPair>(0, dev, grid_for(a.raster, groups), tmH, tmW, a, ep, s) != cudaSuccess)
+  if (launch_one<ProbFwd>(0, dev, grid_for(a.raster, groups), tmH, tmW, tmH, a, status, ep, s) != cudaSuccess)
     return KD_ERR_CUDA;
 
   lse_merge_kernel<<<(unsigned)L.n_merge_blocks, kMergeThreads, 0, s>>>(
@@ -291,11 +314,28 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   return cudaGetLastError() == cudaSuccess ? KD_OK : KD_ERR_CUDA;
 }
 
-int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
-                        const float* topk_logit, const float* mask, int64_t N, int64_t d,
-                        int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
-                        const float* grad_loss, void* dH, float* dW, int accumulate_dW,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Records events[i] (if given) before launch i of the backward pass and
+// events[n] after the last one.
+struct LaunchEvents {
+  cudaEvent_t* ev;
+  int64_t n, next;
+  cudaStream_t s;
+  bool mark() {
+    if (!ev) return true;
+    if (next >= n) return false;
+    return cudaEventRecord(ev[next++], s) == cudaSuccess;
+  }
+};
+
+int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+                  int64_t chunk, const float* lse, const float* grad_loss, void* dH, float* dW,
+                  int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream,
+                  void* const* events, int64_t n_events) {
   Layout L;
   int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
                          workspace_bytes, &L);
@@ -303,9 +343,12 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
   if (!dW || !aligned(dW, 16)) return KD_ERR_INVALID_ARG;
   if (N > 0 && (!lse || !dH || !aligned(dH, 16))) return KD_ERR_INVALID_ARG;
   if ((mask && !aligned(mask, 4)) || (grad_loss && !aligned(grad_loss, 4))) return KD_ERR_INVALID_ARG;
+  const int64_t n_chunks = N > 0 ? ceil_div(N, chunk) : 0;
+  if (events && n_events < (N > 0 ? 2 + 2 * n_chunks + 1 : 0)) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
+  LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
 
   if (cudaMemsetAsync(at<Status>(workspace, L.off_status), 0, sizeof(Status), s) != cudaSuccess)
     return KD_ERR_CUDA;
@@ -322,30 +365,33 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
   float* cscale = at<float>(workspace, L.off_scal);
   __nv_bfloat16* dz = at<__nv_bfloat16>(workspace, L.off_dz);
 
+  if (!evs.mark()) return KD_ERR_CUDA;
   teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
       topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+  if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, nullptr, 0, 1, grad_loss, cscale);
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
 
-  CUtensorMap tmHk, tmWk, tmWmn, tmHmn, tmDW;
+  CUtensorMap tmHk, tmWk, tmWmn, tmHmn, tmDH, tmDW;
   if (!make_map(&tmHk, H, d, N, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, GeoP::B_ROWS) ||
       !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, H, d, N, d, 64, BK) ||
-      !make_map(&tmDW, dW, d, V, d, 32, BM, true))
+      !make_map(&tmDH, dH, d, N, d, 64, BM) || !make_map(&tmDW, dW, d, V, d, 32, BM, true))
     return KD_ERR_CUDA;
   const int groups = resident_groups(dev);
 
   for (int64_t c0 = 0; c0 < N; c0 += chunk) {
     const int64_t Cc = (N - c0 < chunk) ? (N - c0) : chunk;
+    // the chunk's dZ: [Cc][ldz] bf16, as the recompute's store target and the
+    // dH GEMM's A (box {64, 128}), and as the dW GEMM's A (box {64, 64})
     CUtensorMap tmZk, tmZmn;
     if (!make_map(&tmZk, dz, L.ldz, Cc, L.ldz, BK, BM) || !make_map(&tmZmn, dz, L.ldz, Cc, L.ldz, 64, BK))
       return KD_ERR_CUDA;
 
     // dZ for the chunk: recompute z = H W^T tile by tile.
-    GemmArgs a3{};
+    ProbArgs a3{};
     a3.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), true);
     a3.num_kb = (int)ceil_div(d, BK);
     a3.a_row0 = (int)c0;
-    a3.status = status;
     EpiDz::Params e3{};
     e3.rows_valid = (int)Cc;
     e3.row0 = (int)c0;
@@ -357,33 +403,55 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
     e3.lse = lse;
     e3.mask = mask;
     e3.cscale = cscale;
-    e3.tm = tmZk;
-    if (launch_gemm<EpiDz, false, false, kPair>(1, dev, grid_for(a3.raster, groups), tmHk, tmWk, a3, e3, s) != cudaSuccess)
+    if (!evs.mark()) return KD_ERR_CUDA;
+    if (launch_one<ProbDz>(1, dev, grid_for(a3.raster, groups), tmHk, tmWk, tmZk, a3, status, e3, s) != cudaSuccess)
       return KD_ERR_CUDA;
 
-    // dH[chunk] = dZ W   (A = dZ, K-major over V; B = W, MN-major over d).
-    GemmArgs a4{};
-    a4.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), true);
-    a4.num_kb = (int)ceil_div(V, BK);
-    a4.status = status;
+    // One launch for both gradient products of the chunk:
+    //   problem 0: dH[chunk] = dZ W      (few long tiles, K = V)
+    //   problem 1: dW (+)= dZ^T H[chunk] (many short tiles, K = chunk)
+    GemmArgs a45{};
+    a45.status = status;
+    a45.prob[0].raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), true);
+    a45.prob[0].num_kb = (int)ceil_div(V, BK);
+    a45.prob[1].raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
+    a45.prob[1].num_kb = (int)ceil_div(Cc, BK);
+    a45.prob[1].b_k0 = (int)c0;
+    balance_second_problem(a45, groups);
     EpiDh::Params e4{};
-    if (!make_map(&e4.tm, static_cast<__nv_bfloat16*>(dH) + c0 * d, d, Cc, d, 64, BM)) return KD_ERR_CUDA;
-    if (launch_gemm<EpiDh, false, true, kPair>(2, dev, grid_for(a4.raster, groups), tmZk, tmWmn, a4, e4, s) != cudaSuccess)
-      return KD_ERR_CUDA;
-
-    // dW (+)= dZ^T H[chunk]   (A = dZ^T, MN-major over V; B = H, MN-major over d).
-    GemmArgs a5{};
-    a5.raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
-    a5.num_kb = (int)ceil_div(Cc, BK);
-    a5.b_k0 = (int)c0;
-    a5.status = status;
+    e4.row0 = (int)c0;
     EpiDw::Params e5{};
-    e5.tm = tmDW;
     e5.accumulate = (accumulate_dW || c0 > 0) ? 1 : 0;
-    if (launch_gemm<EpiDw, true, true, kPair>(3, dev, grid_for(a5.raster, groups), tmZmn, tmHmn, a5, e5, s) != cudaSuccess)
+    if (!evs.mark()) return KD_ERR_CUDA;
+    if (launch_gemm<ProbDh, ProbDw, kPair>(2, dev, groups, tmZk, tmWmn, tmDH, tmZmn, tmHmn, tmDW, a45, e4, e5, s) != cudaSuccess)
       return KD_ERR_CUDA;
   }
+  if (!evs.mark()) return KD_ERR_CUDA;
   return KD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
+                        const float* topk_logit, const float* mask, int64_t N, int64_t d,
+                        int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
+                        const float* grad_loss, void* dH, float* dW, int accumulate_dW,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_impl(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse, grad_loss, dH,
+                       dW, accumulate_dW, workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+int kd_topk_kl_backward_profiled(const void* H, const void* W, const int32_t* topk_idx,
+                                 const float* topk_logit, const float* mask, int64_t N, int64_t d,
+                                 int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
+                                 const float* grad_loss, void* dH, float* dW, int accumulate_dW,
+                                 void* workspace, size_t workspace_bytes, void* stream,
+                                 void* const* events, int64_t n_events) {
+  if (!events) return KD_ERR_INVALID_ARG;
+  return backward_impl(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse, grad_loss, dH,
+                       dW, accumulate_dW, workspace, workspace_bytes, stream, events, n_events);
 }
 
 int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_count) {

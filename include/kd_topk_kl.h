@@ -109,6 +109,23 @@ int kd_topk_kl_backward(const void* H, const void* W,
                         void* dH, float* dW, int accumulate_dW,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Same as kd_topk_kl_backward, and also records CUDA events on `stream`
+ * around every kernel launch, for timing the pass's kernels live without a
+ * profiler.  events[i] (a cudaEvent_t created by the caller) is recorded
+ * just before the i-th launch and events[n] after the last, n being the
+ * number of launches: 2 + 2 * ceil(N / chunk) for N > 0 (teacher prep,
+ * gradient scale, then per chunk the logit recompute into dZ and the joint
+ * dH / dW launch), 0 for N = 0.  n_events must be at least n + 1, else
+ * KD_ERR_INVALID_ARG and nothing is enqueued. */
+int kd_topk_kl_backward_profiled(const void* H, const void* W,
+                                 const int32_t* topk_idx, const float* topk_logit,
+                                 const float* mask,
+                                 int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                                 const float* lse, const float* grad_loss,
+                                 void* dH, float* dW, int accumulate_dW,
+                                 void* workspace, size_t workspace_bytes, void* stream,
+                                 void* const* events, int64_t n_events);
+
 /* Forward pass for callers that cannot allocate device memory.  The paper
  * has no counterpart to this entry point; it exists for callers such as a
  * runtime that owns all device memory and hands out only fixed buffers, a

@@ -50,6 +50,33 @@ int main() {
         if (!check(tile_raster(ceil_div64(V, 128), ceil_div64(d, 256), false), "dw", C, V, d)) return 1;
         cases += 3;
       }
+  // joint launches: every problem-1 unit in exactly one contiguous range,
+  // and no group's total more than one problem-1 unit above the ideal
+  const long U0s[] = {0, 1, 16, 32, 192, 400};
+  const long k0s[] = {1, 45, 501, 3142};
+  const long U1s[] = {0, 1, 12, 9432, 6012};
+  const long k1s[] = {1, 16, 64};
+  for (long U0 : U0s)
+    for (long k0 : k0s)
+      for (long U1 : U1s)
+        for (long k1 : k1s)
+          for (int g : {1, 7, 74, 148}) {
+            int starts[257];
+            balance_ranges(U0, k0, U1, k1, g, starts);
+            if (starts[0] != 0 || starts[g] != U1) { printf("FAIL joint total\n"); return 1; }
+            double ideal = (double)(U0 * k0 + U1 * k1) / g;
+            long worst0 = ((U0 + g - 1) / g) * k0;
+            for (int i = 0; i < g; ++i) {
+              if (starts[i + 1] < starts[i]) { printf("FAIL joint order\n"); return 1; }
+              long n0 = i < U0 ? (U0 - i + g - 1) / g : 0;
+              double tot = (double)(n0 * k0 + (long)(starts[i + 1] - starts[i]) * k1);
+              if (tot > ideal + k1 + 1e-6 && tot > (double)(n0 * k0) + 1e-6 && (double)worst0 < ideal) {
+                printf("FAIL joint balance U0 %ld k0 %ld U1 %ld k1 %ld g %d: %f vs %f\n", U0, k0, U1, k1, g, tot, ideal);
+                return 1;
+              }
+            }
+            ++cases;
+          }
   printf("OK %d\n", cases);
   return 0;
 }
