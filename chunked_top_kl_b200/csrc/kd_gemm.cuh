@@ -32,6 +32,7 @@ constexpr int BN = 256;          // tile columns (TMEM columns per accumulator)
 constexpr int BK = 64;           // bf16 elements per 128-byte swizzle row
 constexpr int UMMA_K = 16;       // K of one tcgen05.mma kind::f16
 constexpr int GEMM_THREADS = 192;
+constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
 constexpr int TMEM_COLS = 512;
 
 // Per-variant tile geometry.  PAIR = false: one CTA computes a 128 x 256 tile
@@ -477,19 +478,19 @@ struct EpiFwd {
   __device__ __forceinline__ void tile(const Params& P, const CUtensorMap*, int, int n, uint32_t taddr,
                                        EpiCtx&) {
 #pragma unroll 1
-    for (int j = 0; j < BN / 32; ++j) {
-      float v[32];
+    for (int j = 0; j < BN / 64; ++j) {
+      float v[64];
       __syncwarp();
-      tmem_ld_32x32b_x32(taddr + j * 32, v);
-      const int c0 = n * BN + j * 32;
-      if (c0 + 32 > P.V) {
+      tmem_ld_32x32b_x64(taddr + j * 64, v);
+      const int c0 = n * BN + j * 64;
+      if (c0 + 64 > P.V) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 64; ++i)
           if (c0 + i >= P.V) v[i] = -INFINITY;
       }
-      if (nidx < c0 + 32) {
+      if (nidx < c0 + 64) {                 // a teacher column in this group (rare)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < 64; ++i) {
           if (c0 + i == nidx) {
             grun += np * v[i];
             ++cur;
@@ -498,15 +499,27 @@ struct EpiFwd {
           }
         }
       }
-      float cm = v[0];
+      // group max (pairwise tree), then the rescaled running sum-exp with
+      // 2^(z log2(e) - m log2(e)): one FFMA and one ex2 per element
+      float t[32];
 #pragma unroll
-      for (int i = 1; i < 32; ++i) cm = fmaxf(cm, v[i]);
-      const float mn = fmaxf(mrun, cm);
+      for (int i = 0; i < 32; ++i) t[i] = fmaxf(v[i], v[i + 32]);
+#pragma unroll
+      for (int w = 16; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+      const float mn = fmaxf(mrun, t[0]);
       if (mn == -INFINITY) continue;
-      float acc = 0.f;
+      const float mb = mn * kLog2e;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc += __expf(v[i] - mn);
-      srun = srun * __expf(mrun - mn) + acc;
+      for (int i = 0; i < 64; i += 4) {
+        a0 += ex2_approx(fmaf(v[i + 0], kLog2e, -mb));
+        a1 += ex2_approx(fmaf(v[i + 1], kLog2e, -mb));
+        a2 += ex2_approx(fmaf(v[i + 2], kLog2e, -mb));
+        a3 += ex2_approx(fmaf(v[i + 3], kLog2e, -mb));
+      }
+      srun = srun * ex2_approx((mrun - mn) * kLog2e) + ((a0 + a1) + (a2 + a3));
       mrun = mn;
     }
   }
@@ -551,14 +564,22 @@ struct EpiDz {
                                        uint32_t taddr, EpiCtx& cx) {
     const bool valid = r < P.rows_valid;
     const int grow = P.row0 + r;
-    float L = 0.f, c = 0.f;
+    // c exp(z - lse) = 2^(z log2(e) - bias) with bias = lse log2(e) - log2(c):
+    // one FFMA and one ex2 per element.  c = 0 (masked token) and rows past
+    // the chunk give bias = +inf, hence exact zeros.
+    // A negative c (negative upstream gradient or mask weight) is applied
+    // as a sign flip of the packed bf16 pair.
+    float bias = INFINITY, c = 0.f;
+    uint32_t sgn = 0u;
     const int32_t* trow = nullptr;
     const float* prow = nullptr;
     int cur = 0, nidx = kSentinel;
     float np = 0.f;
     if (valid) {
-      L = P.lse[grow];
-      c = (P.mask ? P.mask[grow] : 1.f) * (*P.cscale);
+      const float cs = (P.mask ? P.mask[grow] : 1.f) * (*P.cscale);
+      c = fabsf(cs);
+      sgn = cs < 0.f ? 0x80008000u : 0u;
+      bias = P.lse[grow] * kLog2e - log2f(c);
       trow = P.tidx + (size_t)grow * P.Kp;
       prow = P.tp + (size_t)grow * P.Kp;
       cur = lower_bound_row(trow, P.Kp, n * BN);
@@ -568,32 +589,30 @@ struct EpiDz {
 #pragma unroll 1
     for (int j = 0; j < BN / 64; ++j) {
       float v[64];
-      float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
-      float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
       __syncwarp();
-      tmem_ld_32x32b_x32(taddr + j * 64, v0);
-      tmem_ld_32x32b_x32(taddr + j * 64 + 32, v1);
+      tmem_ld_32x32b_x64(taddr + j * 64, v);
       const int c0 = n * BN + j * 64;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) v[i] = __expf(v[i] - L);
-      if (nidx < c0 + 64) {
+      for (int i = 0; i < 64; ++i) v[i] = ex2_approx(fmaf(v[i], kLog2e, -bias));
+      if (nidx < c0 + 64) {                 // a teacher column in this group (rare)
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           if (c0 + i == nidx) {
-            v[i] -= np;
+            v[i] -= c * np;
             ++cur;
             nidx = trow[cur];
             np = prow[cur];
           }
         }
       }
+      if (c0 + 64 > P.V) {                  // last vocabulary tile: zero columns >= V
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (c0 + i >= P.V) v[i] = 0.f;
+      }
       uint32_t w[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float a = (valid && c0 + 2 * i < P.V) ? c * v[2 * i] : 0.f;
-        const float b = (valid && c0 + 2 * i + 1 < P.V) ? c * v[2 * i + 1] : 0.f;
-        w[i] = pack_bf16x2(a, b);
-      }
+      for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]) ^ sgn;
       stage_store(cx, out, c0, cx.row_base, w, false);
     }
   }
@@ -615,11 +634,8 @@ struct EpiDh {
 #pragma unroll 1
     for (int j = 0; j < BN / 64; ++j) {
       float v[64];
-      float (&v0)[32] = *reinterpret_cast<float(*)[32]>(&v[0]);
-      float (&v1)[32] = *reinterpret_cast<float(*)[32]>(&v[32]);
       __syncwarp();
-      tmem_ld_32x32b_x32(taddr + j * 64, v0);
-      tmem_ld_32x32b_x32(taddr + j * 64 + 32, v1);
+      tmem_ld_32x32b_x64(taddr + j * 64, v);
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);

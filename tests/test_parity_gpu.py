@@ -122,6 +122,13 @@ def test_parity_packed_head_config1(kd):
     assert np.all(got["dH"][masked] == 0.0)
 
 
+def test_negative_upstream_gradient(kd):
+    x = workloads.make_inputs(_cfg(300, 72, 1000, 7, T=0.8, mask="drop5", seed=12))
+    ref = _oracle(x, 0.8, grad=-1.7)
+    got = _gpu(kd, x, 0.8, 100, grad=-1.7)
+    _assert_parity(got, ref, "grad=-1.7")
+
+
 def test_chunk_invariance_and_determinism(kd):
     x = workloads.make_inputs(_cfg(300, 72, 1000, 7, T=0.9, mask="drop5", seed=11))
     base = _gpu(kd, x, 0.9, 300)
