@@ -77,17 +77,20 @@ struct GemmArgs {
   Status* status;
 };
 
-// Compile-time description of a problem: its epilogue and operand majorness.
-template <class EpiT, bool AMN, bool BMN>
+// Compile-time description of a problem: its epilogue, operand majorness,
+// and the L2 eviction priority of each operand's loads (L2Hint).
+template <class EpiT, bool AMN, bool BMN, int AH = kL2Normal, int BH = kL2Normal>
 struct Prob {
   using Epi = EpiT;
   static constexpr bool A_MN = AMN, B_MN = BMN, present = true;
+  static constexpr int A_HINT = AH, B_HINT = BH;
 };
 
 struct EpiNone;
 struct NoProb {
   using Epi = EpiNone;
   static constexpr bool A_MN = false, B_MN = false, present = false;
+  static constexpr int A_HINT = kL2Normal, B_HINT = kL2Normal;
 };
 
 // Loads one operand tile (rows x BK) for K block kb into shared memory.
@@ -97,15 +100,15 @@ struct NoProb {
 //           K-rows of 128 B (64 MN elements); boxes are BK*128 B apart (LBO).
 template <bool MN_MAJOR, int ROWS, bool PAIR>
 __device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* tm, int row, int k,
-                                             uint32_t bar) {
+                                             uint32_t bar, uint64_t policy) {
   if constexpr (!MN_MAJOR) {
-    if constexpr (PAIR) tma_load_2d_pair(dst, tm, k, row, bar);
-    else tma_load_2d(dst, tm, k, row, bar);
+    if constexpr (PAIR) tma_load_2d_pair_hint(dst, tm, k, row, bar, policy);
+    else tma_load_2d_hint(dst, tm, k, row, bar, policy);
   } else {
 #pragma unroll
     for (int i = 0; i < ROWS / 64; ++i) {
-      if constexpr (PAIR) tma_load_2d_pair(dst + i * (BK * 128), tm, row + 64 * i, k, bar);
-      else tma_load_2d(dst + i * (BK * 128), tm, row + 64 * i, k, bar);
+      if constexpr (PAIR) tma_load_2d_pair_hint(dst + i * (BK * 128), tm, row + 64 * i, k, bar, policy);
+      else tma_load_2d_hint(dst + i * (BK * 128), tm, row + 64 * i, k, bar, policy);
     }
   }
 }
@@ -138,7 +141,8 @@ struct EpiCtx {
 // buffer with the 128-byte swizzle, then one thread stores (or adds) the
 // 128-row box to global memory at (x, y) with TMA.
 __device__ __forceinline__ void stage_store(EpiCtx& cx, const CUtensorMap* tm, int x, int y,
-                                            const uint32_t (&w)[32], bool reduce_add) {
+                                            const uint32_t (&w)[32], bool reduce_add,
+                                            int hint = kL2Normal) {
   const uint32_t buf = cx.stage[cx.seq & 1u];
   if (cx.issuer && cx.seq >= 2) bulk_wait_read<1>();     // buffer's previous store has read it
   epilogue_bar_sync(128);
@@ -150,8 +154,9 @@ __device__ __forceinline__ void stage_store(EpiCtx& cx, const CUtensorMap* tm, i
   fence_proxy_async_shared();
   epilogue_bar_sync(128);
   if (cx.issuer) {
-    if (reduce_add) tma_reduce_add_2d(tm, x, y, buf);
-    else tma_store_2d(tm, x, y, buf);
+    const uint64_t pol = make_l2_policy(hint);
+    if (reduce_add) tma_reduce_add_2d_hint(tm, x, y, buf, pol);
+    else tma_store_2d_hint(tm, x, y, buf, pol);
     bulk_commit();
   }
   ++cx.seq;
@@ -274,9 +279,9 @@ __device__ __forceinline__ bool produce_unit(const Smem<G>& L, RoleState& st, ui
       const uint32_t fb = PAIR ? mapa_shared(L.full(st.stage), 0) : L.full(st.stage);
       if (rank == 0) mbar_arrive_expect_tx(L.full(st.stage), G::TX_BYTES);
       load_operand<P::A_MN, BM, PAIR>(sa, tA, pa.a_row0 + m * G::TILE_M + (int)rank * BM,
-                                      pa.a_k0 + kb * BK, fb);
+                                      pa.a_k0 + kb * BK, fb, make_l2_policy(P::A_HINT));
       load_operand<P::B_MN, G::B_ROWS, PAIR>(sb, tB, pa.b_row0 + n * BN + (int)rank * G::B_ROWS,
-                                             pa.b_k0 + kb * BK, fb);
+                                             pa.b_k0 + kb * BK, fb, make_l2_policy(P::B_HINT));
       if (++st.stage == G::STAGES) { st.stage = 0; st.phase ^= 1u; }
     }
   }
@@ -665,7 +670,7 @@ struct EpiDw {
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
-      stage_store(cx, out, n * BN + j * 32, cx.row_base, w, P.accumulate != 0);
+      stage_store(cx, out, n * BN + j * 32, cx.row_base, w, P.accumulate != 0, kL2EvictFirst);
     }
   }
 };

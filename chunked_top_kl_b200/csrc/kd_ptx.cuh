@@ -82,6 +82,28 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int3
       ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar) : "memory");
 }
 
+// L2 eviction-priority policies for the cache-hinted bulk copies below.
+enum L2Hint : int { kL2Normal = 0, kL2EvictFirst = 1, kL2EvictLast = 2 };
+
+__device__ __forceinline__ uint64_t make_l2_policy(int hint) {
+  uint64_t p;
+  if (hint == kL2EvictFirst)
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  else if (hint == kL2EvictLast)
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar), "l"(policy) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -241,6 +263,14 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap,
       ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster_addr) : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                                      uint32_t bar_cluster_addr, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster_addr), "l"(policy) : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
                ::"r"(dst_smem), "r"(ncols) : "memory");
@@ -291,6 +321,19 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, int32_t x, int32_
 __device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, int32_t x, int32_t y, uint32_t src) {
   asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];"
                ::"l"(tmap), "r"(x), "r"(y), "r"(src) : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d_hint(const void* tmap, int32_t x, int32_t y, uint32_t src,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;"
+               ::"l"(tmap), "r"(x), "r"(y), "r"(src), "l"(policy) : "memory");
+}
+
+__device__ __forceinline__ void tma_reduce_add_2d_hint(const void* tmap, int32_t x, int32_t y, uint32_t src,
+                                                       uint64_t policy) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;"
+      ::"l"(tmap), "r"(x), "r"(y), "r"(src), "l"(policy) : "memory");
 }
 
 __device__ __forceinline__ void bulk_commit() {

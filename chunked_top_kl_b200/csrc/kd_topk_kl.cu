@@ -214,10 +214,13 @@ int resident_groups(int dev) {
 
 inline int grid_for(const Raster& r, int groups) { return r.num_units < groups ? r.num_units : groups; }
 
-using ProbFwd = Prob<EpiFwd, false, false>;   // A = H (K-major), B = W (K-major)
-using ProbDz = Prob<EpiDz, false, false>;     // A = H chunk, B = W
+// Operands and their L2 priority: a band of H is re-read for every vocabulary
+// tile of its unit (keep it); the H chunk is re-read by every dW tile of the
+// chunk (keep it); streamed operands use the default priority.
+using ProbFwd = Prob<EpiFwd, false, false, kL2EvictLast, kL2Normal>;  // A = H (K-major), B = W (K-major)
+using ProbDz = Prob<EpiDz, false, false, kL2EvictLast, kL2Normal>;    // A = H chunk, B = W
 using ProbDh = Prob<EpiDh, false, true>;      // A = dZ (K-major over V), B = W (MN-major over d)
-using ProbDw = Prob<EpiDw, true, true>;       // A = dZ^T (MN-major over V), B = H chunk (MN-major over d)
+using ProbDw = Prob<EpiDw, true, true, kL2Normal, kL2EvictLast>;      // A = dZ^T (MN-major over V), B = H chunk
 
 int common_checks(const void* H, const void* W, const int32_t* idx, const float* logit,
                   int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
