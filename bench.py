@@ -1,11 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of the fused chunked top-K KL loss (forward + backward) on B200.
 
-One step = one forward and one backward pass of the whole path over one
-batch of synthetic inputs (teacher-cache preparation, logits + online
-log-sum-exp + teacher gather, lse merge and loss, then per chunk the logit
-recompute into dZ, dH = dZ W and dW += dZ^T H).  Inputs are resident in HBM
-before the timed region starts.
+One step = one fused forward+backward call of the whole path over one batch
+of synthetic inputs (teacher-cache preparation, logits + online log-sum-exp
++ teacher gather, lse merge and loss, then per chunk the logit recompute
+into dZ and the joint dH = dZ W / dW += dZ^T H launch).  Inputs are resident
+in HBM before the timed region starts.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--N TOKENS]
   python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host
@@ -162,32 +162,30 @@ def barrier(world: int):
 
 
 def launches_per_step(N: int, chunk: int) -> int:
-    """Kernels this library launches for one forward + one backward call:
-    forward = teacher prep, logits/lse GEMM, lse merge, finalize;
-    backward = teacher prep, gradient scale, and per chunk the dZ recompute
-    GEMM and the joint dH/dW GEMM."""
+    """Kernels this library launches for one fused forward+backward call:
+    teacher prep, logits/lse GEMM, lse merge, loss, gradient scale, and per
+    chunk the dZ recompute GEMM and the joint dH/dW GEMM."""
     if N == 0:
         return 0
-    return 4 + 2 + 2 * math.ceil(N / chunk)
+    return 5 + 2 * math.ceil(N / chunk)
 
 
-def per_kernel_times(ev_b, ev_f, N, d, V, chunk):
-    """Live per-kernel totals from the events recorded around every backward
-    launch (launch 0 teacher prep, 1 gradient scale, then per chunk c the
-    dZ recompute 2+2c and the joint dH/dW GEMM 3+2c) and around the forward
-    call (its GEMM plus three sub-0.2 ms kernels)."""
-    steps = len(ev_b)
-    out = {"forward_gemm": {"launches": steps, "ms": sum(a.elapsed_time(b) for a, b in ev_f),
-                            "flops": 2.0 * N * d * V * steps}}
-    names = {0: "teacher_prep", 1: "grad_scale"}
-    for row in ev_b:
+def per_kernel_times(ev, N, d, V, chunk):
+    """Live per-kernel totals from the events recorded around every launch of
+    the fused call: 0 teacher prep, 1 logits/lse GEMM, 2 lse merge, 3 loss,
+    4 gradient scale, then per chunk c the dZ recompute (5+2c) and the joint
+    dH/dW GEMM (6+2c)."""
+    names = {0: ("teacher_prep", 0.0), 1: ("forward_gemm", 2.0 * N * d * V), 2: ("lse_merge", 0.0),
+             3: ("loss", 0.0), 4: ("grad_scale", 0.0)}
+    out = {}
+    for row in ev:
         for j in range(len(row) - 1):
             if j in names:
-                key, flops = names[j], 0.0
+                key, flops = names[j]
             else:
-                c = (j - 2) // 2
+                c = (j - 5) // 2
                 cc = min(chunk, N - c * chunk)
-                key, flops = (("dz_recompute", 2.0 * cc * d * V) if j % 2 == 0
+                key, flops = (("dz_recompute", 2.0 * cc * d * V) if (j - 5) % 2 == 0
                               else ("grads_dH_dW", 4.0 * cc * d * V))
             k = out.setdefault(key, {"launches": 0, "ms": 0.0, "flops": 0.0})
             k["launches"] += 1
@@ -280,9 +278,8 @@ def run_cuda(args, cfg, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, workspace=ws)
-        kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, lse,
-                    workspace=ws, dH=dH, dW=dW)
+        loss, _, _, _ = kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T,
+                                            chunk, workspace=ws, dH=dH, dW=dW)
         return loss
 
     for _ in range(args.warmup):
@@ -294,15 +291,15 @@ def run_cuda(args, cfg, world, rank, local):
     peak_gib = (torch.cuda.max_memory_allocated(dev) - base_mem) / 2**30
     ws_gib = ws.numel() / 2**30
 
-    # ---- kernel-only timed region (inputs resident in HBM).  The backward
-    # pass records an event around each of its kernel launches (same kernels
-    # and work as the plain call), which gives live per-kernel durations.
-    nl = kd.backward_launches(N, chunk)
-    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    ev_b = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(args.steps)]
-    for e in [x for pair in ev_f for x in pair] + [x for row in ev_b for x in row]:
-        e.record(stream)                     # creates the CUDA event behind each object
+    # ---- kernel-only timed region (inputs resident in HBM).  Each step is one
+    # fused forward+backward call that records an event before each of its
+    # kernel launches and after the last (same kernels and work as without
+    # events), which gives live per-kernel durations on the launching stream.
+    nl = kd.forward_backward_launches(N, chunk)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)                 # creates the CUDA event behind each object
     sampler = ClockSampler(local) if not args.no_clocks else None
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -313,19 +310,14 @@ def run_cuda(args, cfg, world, rank, local):
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        ev_f[i][0].record(stream)
-        loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, workspace=ws)
-        ev_f[i][1].record(stream)
-        kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, lse,
-                    workspace=ws, dH=dH, dW=dW, events=ev_b[i])
+        kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk,
+                            workspace=ws, dH=dH, dW=dW, events=ev[i])
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     clocks = sampler.stop() if sampler else None
     ms_local = start.elapsed_time(end)
-    fwd_ms = [a.elapsed_time(b) for a, b in ev_f]
-    bwd_ms = [row[0].elapsed_time(row[-1]) for row in ev_b]
-    kern = per_kernel_times(ev_b, ev_f, N, d, V, chunk)
+    kern = per_kernel_times(ev, N, d, V, chunk)
     ms = reduce_max(ms_local, world, dev)
     st, _ = kd.check(ws)
     if st != 0:
@@ -370,8 +362,8 @@ def run_cuda(args, cfg, world, rank, local):
     # Roofline of the dominant kernel (largest share of the step's kernel time).
     dom_name, dom = max(((k, v) for k, v in kern.items() if v["flops"] > 0), key=lambda kv: kv[1]["ms"])
     dom_ach = dom["tflops"]
-    fwd_avg = sum(fwd_ms) / len(fwd_ms)
-    bwd_avg = sum(bwd_ms) / len(bwd_ms)
+    fwd_avg = sum(kern[k]["ms"] for k in ("teacher_prep", "forward_gemm", "lse_merge", "loss")) / args.steps
+    bwd_avg = sum(kern[k]["ms"] for k in ("grad_scale", "dz_recompute", "grads_dH_dW")) / args.steps
     peak_sus = peaks["bf16_tflops_sustained"]
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

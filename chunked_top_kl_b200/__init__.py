@@ -9,13 +9,15 @@ been built; there is no fallback path.
 
 from ._abi import (EXPORTS, KDError, kd_status_string, kd_topk_kl_backward,
                    kd_topk_kl_backward_profiled, kd_topk_kl_check, kd_topk_kl_forward,
-                   kd_topk_kl_forward_noalloc, kd_topk_kl_workspace_size, load)
+                   kd_topk_kl_forward_backward, kd_topk_kl_forward_noalloc, kd_topk_kl_workspace_size,
+                   load)
 from .api import (KDTopKKLFunction, alloc_workspace, backward, backward_launches, check, forward,
-                  kd_topk_kl_loss, workspace_bytes)
+                  forward_backward, forward_backward_launches, kd_topk_kl_loss, workspace_bytes)
 
 __all__ = [
     "EXPORTS", "KDError", "kd_status_string", "kd_topk_kl_backward", "kd_topk_kl_backward_profiled",
     "kd_topk_kl_check",
     "kd_topk_kl_forward", "kd_topk_kl_forward_noalloc", "kd_topk_kl_workspace_size", "KDTopKKLFunction", "alloc_workspace",
-    "backward", "backward_launches", "check", "forward", "kd_topk_kl_loss", "workspace_bytes",
+    "backward", "backward_launches", "check", "forward", "forward_backward", "forward_backward_launches",
+    "kd_topk_kl_forward_backward", "kd_topk_kl_loss", "workspace_bytes",
 ]

@@ -28,6 +28,7 @@ EXPORTS = (
     "kd_topk_kl_check",
     "kd_topk_kl_forward_noalloc",
     "kd_topk_kl_backward_profiled",
+    "kd_topk_kl_forward_backward",
 )
 
 _lib = None
@@ -56,6 +57,9 @@ def load() -> ctypes.CDLL:
         lib.kd_topk_kl_backward_profiled.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p,
                                                      p, i32, p, sz, p, ctypes.POINTER(ctypes.c_void_p), i64]
         lib.kd_topk_kl_backward_profiled.restype = i32
+        lib.kd_topk_kl_forward_backward.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p, p, p,
+                                                    i32, p, sz, p, ctypes.POINTER(ctypes.c_void_p), i64]
+        lib.kd_topk_kl_forward_backward.restype = i32
         lib.kd_topk_kl_forward_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, p, p, p]
         lib.kd_topk_kl_forward_noalloc.restype = i32
         _lib = lib
@@ -98,6 +102,21 @@ def kd_topk_kl_backward_profiled(H, W, topk_idx, topk_logit, mask, N, d, V, K, T
     return int(load().kd_topk_kl_backward_profiled(H, W, topk_idx, topk_logit, mask, N, d, V, K, T,
                                                    chunk, lse, grad_loss, dH, dW, int(accumulate_dW),
                                                    workspace, workspace_bytes, stream, arr, len(events)))
+
+
+def kd_topk_kl_forward_backward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, loss, lse,
+                                grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes, stream,
+                                events=None) -> int:
+    """``events``: None, or cudaEvent_t handles (ints), one more than the
+    call's launches (5 + 2 * ceil(N / chunk))."""
+    if events:
+        arr = (ctypes.c_void_p * len(events))(*events)
+        n = len(events)
+    else:
+        arr, n = None, 0
+    return int(load().kd_topk_kl_forward_backward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk,
+                                                  loss, lse, grad_loss, dH, dW, int(accumulate_dW),
+                                                  workspace, workspace_bytes, stream, arr, n))
 
 
 def kd_topk_kl_check(workspace, stream) -> tuple[int, int]:

@@ -109,6 +109,39 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
     return dH, dW
 
 
+def forward_backward_launches(N: int, chunk: int) -> int:
+    """Kernel launches of one fused forward + backward call."""
+    return 0 if N == 0 else 5 + 2 * ((N + chunk - 1) // chunk)
+
+
+def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
+                     grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
+                     accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
+                     dH: Optional[torch.Tensor] = None, events=None):
+    """One call for a training step: returns (loss, lse, dH, dW)."""
+    N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
+    dev = H.device
+    if workspace is None:
+        workspace = alloc_workspace(N, d, V, K, chunk, dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    if dH is None:
+        dH = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    if dW is None:
+        dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+        accumulate_dW = False
+    if grad_loss is not None:
+        grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = _abi.kd_topk_kl_forward_backward(
+        _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T), int(chunk),
+        _ptr(loss), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+        _ptr(workspace), workspace.numel(), stream,
+        None if events is None else [e.cuda_event for e in events])
+    _raise(st, "kd_topk_kl_forward_backward")
+    return loss, lse, dH, dW
+
+
 def check(workspace: torch.Tensor) -> Tuple[int, int]:
     """Synchronise the current stream and read the device status words:
     returns (status, bad_index_count)."""

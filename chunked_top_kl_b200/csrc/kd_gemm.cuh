@@ -31,7 +31,7 @@ constexpr int BM = 128;          // accumulator rows per CTA (TMEM lanes)
 constexpr int BN = 256;          // tile columns (TMEM columns per accumulator)
 constexpr int BK = 64;           // bf16 elements per 128-byte swizzle row
 constexpr int UMMA_K = 16;       // K of one tcgen05.mma kind::f16
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 192;   // warps: 0 TMA, 1 MMA, 2-5 epilogue
 constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
 constexpr int TMEM_COLS = 512;
 

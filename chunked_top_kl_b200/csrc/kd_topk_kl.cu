@@ -239,6 +239,25 @@ int common_checks(const void* H, const void* W, const int32_t* idx, const float*
 template <class T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
 
+// Records events[i] (if given) before the i-th kernel launch of a call and
+// events[n] after the last one.
+struct LaunchEvents {
+  cudaEvent_t* ev;
+  int64_t n, next;
+  cudaStream_t s;
+  bool mark() {
+    if (!ev) return true;
+    if (next >= n) return false;
+    return cudaEventRecord(ev[next++], s) == cudaSuccess;
+  }
+};
+
+
+int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+                  const Layout& L, float* loss, float* lse, void* workspace, cudaStream_t s,
+                  LaunchEvents& evs);
+
 }  // namespace
 
 extern "C" {
@@ -272,6 +291,20 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   if (!loss || (N > 0 && !lse)) return KD_ERR_INVALID_ARG;
   if (mask && !aligned(mask, 4)) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LaunchEvents evs{nullptr, 0, 0, s};
+  return forward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, L, loss, lse, workspace, s, evs);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Forward pass on a checked workspace layout: clears the status words, then
+// teacher prep, the logits/lse GEMM, the lse merge and the loss.
+int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+                  const Layout& L, float* loss, float* lse, void* workspace, cudaStream_t s,
+                  LaunchEvents& evs) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
 
@@ -287,6 +320,7 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   double* mask_part = at<double>(workspace, L.off_mask_part);
   double* term_part = at<double>(workspace, L.off_term_part);
 
+  if (!evs.mark()) return KD_ERR_CUDA;
   teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
       topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
@@ -307,53 +341,40 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
   ep.part_m = at<float>(workspace, L.off_pm);
   ep.part_s = at<float>(workspace, L.off_ps);
   ep.part_g = at<float>(workspace, L.off_pg);
+  if (!evs.mark()) return KD_ERR_CUDA;
   if (launch_one<ProbFwd>(0, dev, grid_for(a.raster, groups), tmH, tmW, tmH, a, status, ep, s) != cudaSuccess)
     return KD_ERR_CUDA;
 
+  if (!evs.mark()) return KD_ERR_CUDA;
   lse_merge_kernel<<<(unsigned)L.n_merge_blocks, kMergeThreads, 0, s>>>(
       ep.part_m, ep.part_s, ep.part_g, a.raster.splits, (int)N, ent, mask, lse, term_part);
+  if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, term_part,
                                     (int)L.n_merge_blocks, 0, nullptr, loss);
   return cudaGetLastError() == cudaSuccess ? KD_OK : KD_ERR_CUDA;
 }
 
-}  // extern "C"
 
-namespace {
-
-// Records events[i] (if given) before launch i of the backward pass and
-// events[n] after the last one.
-struct LaunchEvents {
-  cudaEvent_t* ev;
-  int64_t n, next;
-  cudaStream_t s;
-  bool mark() {
-    if (!ev) return true;
-    if (next >= n) return false;
-    return cudaEventRecord(ev[next++], s) == cudaSuccess;
-  }
-};
-
-int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
-                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
-                  int64_t chunk, const float* lse, const float* grad_loss, void* dH, float* dW,
-                  int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream,
-                  void* const* events, int64_t n_events) {
-  Layout L;
-  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
-                         workspace_bytes, &L);
-  if (st != KD_OK) return st;
+int backward_checks(int64_t N, const float* lse, const float* grad_loss, const float* mask,
+                    const void* dH, const float* dW) {
   if (!dW || !aligned(dW, 16)) return KD_ERR_INVALID_ARG;
   if (N > 0 && (!lse || !dH || !aligned(dH, 16))) return KD_ERR_INVALID_ARG;
   if ((mask && !aligned(mask, 4)) || (grad_loss && !aligned(grad_loss, 4))) return KD_ERR_INVALID_ARG;
-  const int64_t n_chunks = N > 0 ? ceil_div(N, chunk) : 0;
-  if (events && n_events < (N > 0 ? 2 + 2 * n_chunks + 1 : 0)) return KD_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return KD_OK;
+}
+
+// Backward pass on a checked workspace layout.  With run_prep the status
+// words are cleared and the teacher cache is prepared here; without it the
+// forward pass of the same call has done both.  Then the gradient scale and,
+// per chunk, the dZ recompute and the joint dH / dW launch.
+int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
+                   const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+                   int64_t chunk, const Layout& L, const float* lse, const float* grad_loss,
+                   void* dH, float* dW, int accumulate_dW, void* workspace, cudaStream_t s,
+                   bool run_prep, LaunchEvents& evs) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
-  LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
-
-  if (cudaMemsetAsync(at<Status>(workspace, L.off_status), 0, sizeof(Status), s) != cudaSuccess)
+  if (run_prep && cudaMemsetAsync(at<Status>(workspace, L.off_status), 0, sizeof(Status), s) != cudaSuccess)
     return KD_ERR_CUDA;
   if (N == 0) {
     if (!accumulate_dW && cudaMemsetAsync(dW, 0, sizeof(float) * (size_t)V * d, s) != cudaSuccess)
@@ -368,9 +389,11 @@ int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const f
   float* cscale = at<float>(workspace, L.off_scal);
   __nv_bfloat16* dz = at<__nv_bfloat16>(workspace, L.off_dz);
 
-  if (!evs.mark()) return KD_ERR_CUDA;
-  teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
-      topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+  if (run_prep) {
+    if (!evs.mark()) return KD_ERR_CUDA;
+    teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
+        topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+  }
   if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, nullptr, 0, 1, grad_loss, cscale);
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
@@ -429,7 +452,6 @@ int backward_impl(const void* H, const void* W, const int32_t* topk_idx, const f
     if (launch_gemm<ProbDh, ProbDw, kPair>(2, dev, groups, tmZk, tmWmn, tmDH, tmZmn, tmHmn, tmDW, a45, e4, e5, s) != cudaSuccess)
       return KD_ERR_CUDA;
   }
-  if (!evs.mark()) return KD_ERR_CUDA;
   return KD_OK;
 }
 
@@ -442,8 +464,9 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
                         int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
                         const float* grad_loss, void* dH, float* dW, int accumulate_dW,
                         void* workspace, size_t workspace_bytes, void* stream) {
-  return backward_impl(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse, grad_loss, dH,
-                       dW, accumulate_dW, workspace, workspace_bytes, stream, nullptr, 0);
+  return kd_topk_kl_backward_profiled(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse,
+                                      grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes,
+                                      stream, nullptr, 0);
 }
 
 int kd_topk_kl_backward_profiled(const void* H, const void* W, const int32_t* topk_idx,
@@ -452,9 +475,43 @@ int kd_topk_kl_backward_profiled(const void* H, const void* W, const int32_t* to
                                  const float* grad_loss, void* dH, float* dW, int accumulate_dW,
                                  void* workspace, size_t workspace_bytes, void* stream,
                                  void* const* events, int64_t n_events) {
-  if (!events) return KD_ERR_INVALID_ARG;
-  return backward_impl(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse, grad_loss, dH,
-                       dW, accumulate_dW, workspace, workspace_bytes, stream, events, n_events);
+  Layout L;
+  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
+                         workspace_bytes, &L);
+  if (st != KD_OK) return st;
+  if ((st = backward_checks(N, lse, grad_loss, mask, dH, dW)) != KD_OK) return st;
+  const int64_t launches = N > 0 ? 2 + 2 * ceil_div(N, chunk) : 0;
+  if (events && n_events < launches + 1) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
+  st = backward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, L, lse, grad_loss, dH,
+                      dW, accumulate_dW, workspace, s, true, evs);
+  if (st == KD_OK && N > 0 && !evs.mark()) return KD_ERR_CUDA;
+  return st;
+}
+
+int kd_topk_kl_forward_backward(const void* H, const void* W, const int32_t* topk_idx,
+                                const float* topk_logit, const float* mask, int64_t N, int64_t d,
+                                int64_t V, int64_t K, float T, int64_t chunk, float* loss,
+                                float* lse, const float* grad_loss, void* dH, float* dW,
+                                int accumulate_dW, void* workspace, size_t workspace_bytes,
+                                void* stream, void* const* events, int64_t n_events) {
+  Layout L;
+  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
+                         workspace_bytes, &L);
+  if (st != KD_OK) return st;
+  if (!loss || (N > 0 && !lse)) return KD_ERR_INVALID_ARG;
+  if ((st = backward_checks(N, lse, grad_loss, mask, dH, dW)) != KD_OK) return st;
+  const int64_t launches = N > 0 ? 5 + 2 * ceil_div(N, chunk) : 0;
+  if (events && n_events < launches + 1) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
+  st = forward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, L, loss, lse, workspace, s, evs);
+  if (st != KD_OK) return st;
+  st = backward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, L, lse, grad_loss, dH,
+                      dW, accumulate_dW, workspace, s, false, evs);
+  if (st == KD_OK && N > 0 && !evs.mark()) return KD_ERR_CUDA;
+  return st;
 }
 
 int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_count) {

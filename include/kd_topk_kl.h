@@ -126,6 +126,23 @@ int kd_topk_kl_backward_profiled(const void* H, const void* W,
                                  void* workspace, size_t workspace_bytes, void* stream,
                                  void* const* events, int64_t n_events);
 
+/* Forward and backward pass in one call, for a training step whose loss is
+ * this one: writes *loss and lse[N] as kd_topk_kl_forward, then dH and dW as
+ * kd_topk_kl_backward (grad_loss as there; NULL for 1.0).  The teacher cache
+ * is prepared once for both passes.  events may be NULL; otherwise it holds
+ * cudaEvent_t handles recorded on `stream` before each kernel launch and
+ * after the last: n = 5 + 2 * ceil(N / chunk) launches for N > 0 (teacher
+ * prep, logits/lse GEMM, lse merge, loss, gradient scale, then per chunk the
+ * dZ recompute and the joint dH / dW launch), n_events >= n + 1. */
+int kd_topk_kl_forward_backward(const void* H, const void* W,
+                                const int32_t* topk_idx, const float* topk_logit,
+                                const float* mask,
+                                int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                                float* loss, float* lse, const float* grad_loss,
+                                void* dH, float* dW, int accumulate_dW,
+                                void* workspace, size_t workspace_bytes, void* stream,
+                                void* const* events, int64_t n_events);
+
 /* Forward pass for callers that cannot allocate device memory.  The paper
  * has no counterpart to this entry point; it exists for callers such as a
  * runtime that owns all device memory and hands out only fixed buffers, a

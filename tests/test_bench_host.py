@@ -46,8 +46,8 @@ def test_launch_count_and_config_block():
     sys.path.insert(0, ROOT)
     import bench
     import workloads
-    assert bench.launches_per_step(32768, 4096) == 6 + 2 * 8
-    assert bench.launches_per_step(300, 128) == 6 + 2 * 3
+    assert bench.launches_per_step(32768, 4096) == 5 + 2 * 8
+    assert bench.launches_per_step(300, 128) == 5 + 2 * 3
     assert bench.launches_per_step(0, 128) == 0
     blk = bench.config_block(workloads.get_config(3), 4)
     assert blk["global_batch"] == 4 * 32768 and blk["workload"].startswith("gptoss_head")

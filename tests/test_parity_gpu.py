@@ -223,3 +223,48 @@ def test_autograd_wrapper(kd):
     assert abs(loss.item() - ref["loss"]) / ref["loss"] <= LOSS_RTOL
     assert _rfro(H.grad.float().cpu().double().numpy(), ref["dH"]) <= GRAD_RFRO
     assert _rfro(W.grad.float().cpu().double().numpy(), ref["dW"]) <= GRAD_RFRO
+
+
+def test_fused_forward_backward_matches_separate_calls(kd):
+    for (N, d, V, K, T, chunk) in [(300, 72, 1000, 7, 0.7, 100), (512, 256, 4096, 16, 1.0, 128)]:
+        x = workloads.make_inputs(_cfg(N, d, V, K, T=T, mask="drop5", seed=13))
+        g = _to_dev(x)
+        ws = kd.alloc_workspace(N, d, V, K, chunk, "cuda")
+        gl = torch.tensor(1.3, device="cuda")
+        loss_a, lse_a = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, workspace=ws)
+        dH_a, dW_a = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk, lse_a,
+                                 grad_loss=gl, workspace=ws)
+        n = kd.forward_backward_launches(N, chunk)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        for e in ev:
+            e.record()
+        loss_b, lse_b, dH_b, dW_b = kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"],
+                                                         g["mask"], T, chunk, grad_loss=gl, workspace=ws,
+                                                         events=ev)
+        torch.cuda.synchronize()
+        assert kd.check(ws) == (0, 0)
+        assert loss_a.item() == loss_b.item()
+        assert torch.equal(lse_a, lse_b) and torch.equal(dH_a, dH_b) and torch.equal(dW_a, dW_b)
+        times = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+        assert all(t >= 0 for t in times)
+        ref = _oracle(x, T, grad=1.3)
+        _assert_parity({"loss": loss_b.item(), "lse": lse_b.cpu().double().numpy(),
+                        "dH": dH_b.float().cpu().double().numpy(), "dW": dW_b.cpu().double().numpy()},
+                       ref, f"fused {N}")
+
+
+def test_event_count_is_checked(kd):
+    x = workloads.make_inputs(_cfg(200, 64, 700, 6, seed=14))
+    g = _to_dev(x)
+    ws = kd.alloc_workspace(200, 64, 700, 6, 64, "cuda")
+    _, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws)
+    n = kd.backward_launches(200, 64)
+    too_few = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in too_few:
+        e.record()
+    with pytest.raises(kd.KDError):
+        kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, lse, workspace=ws,
+                    events=too_few)
+    with pytest.raises(kd.KDError):
+        kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws,
+                            events=too_few)
