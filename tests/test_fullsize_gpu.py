@@ -1,5 +1,5 @@
 """Parity at the full workload sizes, in the launch configuration bench.py
-times (same chunk, same entry points).
+times (same chunk, the same fused forward + backward entry point).
 
 Expected values come from ``tests/golden/fullsize_*.npz``, written by
 ``tests/golden/make_fullsize_expected.py`` with the fp64 oracle only: the
@@ -71,10 +71,8 @@ def test_fullsize_parity(kd, path):
 
     g = {k: v.cuda() for k, v in x.items()}
     ws = kd.alloc_workspace(cfg.N, cfg.d, cfg.V, cfg.K, cfg.chunk, "cuda")
-    loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], cfg.T, cfg.chunk,
-                           workspace=ws)
-    dH, dW = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], cfg.T, cfg.chunk,
-                         lse, workspace=ws)
+    loss, lse, dH, dW = kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], cfg.T,
+                                            cfg.chunk, workspace=ws)
     st, nbad = kd.check(ws)
     assert st == 0, kd.kd_status_string(st)
 
