@@ -55,8 +55,6 @@ struct Geo {
   static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // per stage, whole tile
 };
 
-constexpr int kMaxGroups = 160;   // >= resident CTAs (or CTA pairs) on one GPU
-
 // One GEMM as the kernel sees it: its tile schedule, K blocks per tile, and
 // offsets added to the tensor-map coordinates of A and B.
 struct ProbArgs {
@@ -67,13 +65,12 @@ struct ProbArgs {
 };
 
 // A launch runs problem 0 and, optionally, problem 1.  Problem 0's units go
-// round-robin over the groups (CTAs, or CTA pairs); problem 1's units are
-// split into one contiguous range per group, [p1_start[g], p1_start[g+1]),
-// sized on the host so that every group gets about the same number of K
-// blocks in total.  Every role of a group walks the same sequence.
+// round-robin over the groups (CTAs, or CTA pairs); problem 1's are dealt by
+// `joint` (see joint_plan), so that every group gets about the same number
+// of K blocks in total.  Every role of a group walks the same sequence.
 struct GemmArgs {
   ProbArgs prob[2];
-  int p1_start[kMaxGroups + 1];
+  JointPlan joint;
   Status* status;
 };
 
@@ -398,8 +395,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     for (int u = group; ok && u < args.prob[0].raster.num_units; u += ngroups)
       ok = body(P0{}, args.prob[0], &tmA0, &tmB0, u);
     if constexpr (P1::present) {
-      for (int u = args.p1_start[group]; ok && u < args.p1_start[group + 1]; ++u)
-        ok = body(P1{}, args.prob[1], &tmA1, &tmB1, u);
+      const int n1 = joint_count(args.joint, args.prob[1].raster.num_units, ngroups, group);
+      for (int i = 0; ok && i < n1; ++i)
+        ok = body(P1{}, args.prob[1], &tmA1, &tmB1, joint_unit(args.joint, ngroups, group, i));
     }
     return ok;
   };

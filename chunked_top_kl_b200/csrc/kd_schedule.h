@@ -60,7 +60,14 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
 // running log-sum-exp one CTA carries.  Picks the number of ranges
 // (<= kMaxSplits) minimising waves x tiles-per-unit on `grid` CTAs; every
 // range is non-empty.
-inline Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid) {
+//
+// The B operand (the vocabulary rows) is the large one, so a wave should
+// share each column tile among as many bands as it can: group_m bands walk
+// the same ranges side by side, group_m = grid / 2 (two ranges per wave),
+// capped so the group's A bands (band_bytes each, kept in L2) take at most
+// half of `l2_budget`, and evened out over the groups.
+inline Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid, int64_t band_bytes = 0,
+                             int64_t l2_budget = 0) {
   int best_s = 1;
   int64_t best_cost = INT64_MAX;
   for (int s = 1; s <= kMaxSplits && s <= n_tiles; ++s) {
@@ -74,48 +81,64 @@ inline Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid) {
   r.n_tiles = (int)n_tiles;
   r.tiles_per_split = (int)ceil_div64(n_tiles, best_s);
   r.splits = (int)ceil_div64(n_tiles, r.tiles_per_split);
-  int gm = grid / r.splits;
-  r.group_m = gm < 1 ? 1 : (gm > m_tiles ? (int)m_tiles : gm);
+  int64_t gm = grid / 2;
+  if (band_bytes > 0 && l2_budget > 0) {
+    const int64_t cap = l2_budget / 2 / band_bytes;
+    if (gm > cap) gm = cap;
+  }
+  if (gm < 1) gm = 1;
+  if (gm > m_tiles) gm = m_tiles;
+  gm = ceil_div64(m_tiles, ceil_div64(m_tiles, gm));
+  r.group_m = (int)gm;
   r.num_units = (int)(m_tiles * r.splits);
   return r;
 }
 
-// Two problems in one launch: problem 0's U0 units (k0 K blocks each) go
-// round-robin over `groups`; problem 1's U1 units (k1 K blocks each) are cut
-// into one contiguous range per group, [starts[g], starts[g+1]), sized so
-// that every group's total K blocks are as equal as whole units allow
-// (largest remainders first).  starts has groups + 1 entries.
-inline void balance_ranges(int64_t U0, int64_t k0, int64_t U1, int64_t k1, int groups, int* starts) {
-  const double target = (double)(U0 * k0 + U1 * k1) / groups;
-  int64_t sum = 0;
-  int64_t cnt[256];
-  double frac[256];
-  for (int g = 0; g < groups; ++g) {
-    const int64_t n0 = g < U0 ? (U0 - g + groups - 1) / groups : 0;
-    double want = (target - (double)(n0 * k0)) / (double)(k1 > 0 ? k1 : 1);
-    if (want < 0) want = 0;
-    cnt[g] = (int64_t)want;
-    frac[g] = want - (double)cnt[g];
-    sum += cnt[g];
+// Two problems in one launch.  Problem 0's U0 units (k0 K blocks each) go
+// round-robin over `groups`, so groups [0, r), r = U0 % groups, run one more
+// of them than the others.  Problem 1's U1 units (k1 K blocks each) are dealt
+// so that groups running at the same time hold neighbouring units (which
+// share operand tiles in L2) while every group's K blocks add up to about the
+// same: first the groups >= r, free one problem-0 unit earlier, take
+// wb ~ k0 / k1 units each, round-robin among themselves; then all groups take
+// the rest round-robin, the class with less work so far first.
+struct JointPlan {
+  int r;     // groups [0, r) run one more problem-0 unit
+  int wb;    // problem-1 units each group >= r runs before the others join
+  int p2;    // first problem-1 unit dealt round-robin to all groups
+  int rot;   // group g's place in that round-robin is (g - rot) mod groups
+};
+
+KD_HD JointPlan joint_plan(int64_t U0, int64_t k0, int64_t U1, int64_t k1, int groups) {
+  JointPlan p;
+  p.r = (int)(U0 % groups);
+  const int64_t nb = groups - p.r;
+  int64_t wb = 0;
+  if (p.r > 0 && k1 > 0) {
+    wb = (k0 + k1 / 2) / k1;
+    if (wb > U1 / nb) wb = U1 / nb;
   }
-  while (sum < U1) {
-    int best = 0;
-    for (int g = 1; g < groups; ++g)
-      if (frac[g] > frac[best]) best = g;
-    cnt[best] += 1;
-    frac[best] -= 1.0;
-    sum += 1;
+  p.wb = (int)wb;
+  p.p2 = (int)(wb * nb);
+  p.rot = (wb * k1 <= k0) ? p.r : 0;
+  return p;
+}
+
+// Problem-1 units of group g, and the i-th of them.
+KD_HD int joint_count(const JointPlan& p, int64_t U1, int groups, int g) {
+  const int first = g >= p.r ? p.wb : 0;
+  const int64_t gp = (g - p.rot + groups) % groups;
+  const int64_t left = U1 - p.p2 - gp;
+  return first + (left > 0 ? (int)ceil_div64(left, groups) : 0);
+}
+
+KD_HD int joint_unit(const JointPlan& p, int groups, int g, int i) {
+  if (g >= p.r) {
+    if (i < p.wb) return (g - p.r) + i * (groups - p.r);
+    i -= p.wb;
   }
-  while (sum > U1) {
-    int best = -1;
-    for (int g = 0; g < groups; ++g)
-      if (cnt[g] > 0 && (best < 0 || frac[g] < frac[best])) best = g;
-    cnt[best] -= 1;
-    frac[best] += 1.0;
-    sum -= 1;
-  }
-  starts[0] = 0;
-  for (int g = 0; g < groups; ++g) starts[g + 1] = starts[g] + (int)cnt[g];
+  const int gp = (g - p.rot + groups) % groups;
+  return p.p2 + gp + i * groups;
 }
 
 }  // namespace kd

@@ -114,6 +114,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 struct DevInfo {
   int sms = 0;
   int pair_groups = 0;          // co-resident CTA pairs of the GEMM kernel
+  int64_t l2_bytes = 0;
   bool attr_set[8] = {};
 };
 DevInfo g_dev[kMaxDevices];
@@ -126,6 +127,16 @@ int device_sms(int dev) {
     g_dev[dev].sms = v > 0 ? v : 148;
   }
   return g_dev[dev].sms;
+}
+
+int64_t device_l2_bytes(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return 126ll << 20;
+  if (!g_dev[dev].l2_bytes) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev);
+    g_dev[dev].l2_bytes = v > 0 ? v : (126ll << 20);
+  }
+  return g_dev[dev].l2_bytes;
 }
 
 // All GEMMs run as CTA pairs (cta_group::2, 256 x 256 tiles).
@@ -174,12 +185,12 @@ cudaError_t launch_one(int slot, int dev, int groups, const CUtensorMap& ta, con
   return launch_gemm<P0, NoProb, kPair>(slot, dev, groups, ta, tb, to, ta, tb, to, a, ep, none, s);
 }
 
-// Problem 0 round-robin, problem 1 in contiguous per-group ranges that even
-// out the groups' total K blocks (see balance_ranges).
-void balance_second_problem(GemmArgs& a, int groups) {
-  balance_ranges(a.prob[0].raster.num_units, (int64_t)a.prob[0].raster.tiles_per_split * a.prob[0].num_kb,
-                 a.prob[1].raster.num_units, (int64_t)a.prob[1].raster.tiles_per_split * a.prob[1].num_kb,
-                 groups, a.p1_start);
+// Problem 0 round-robin, problem 1 dealt to even out the groups' total K
+// blocks (see joint_plan).
+void plan_second_problem(GemmArgs& a, int groups) {
+  a.joint = joint_plan(a.prob[0].raster.num_units, (int64_t)a.prob[0].raster.tiles_per_split * a.prob[0].num_kb,
+                       a.prob[1].raster.num_units, (int64_t)a.prob[1].raster.tiles_per_split * a.prob[1].num_kb,
+                       groups);
 }
 
 // Work groups (CTAs, or CTA pairs) that can be resident at once: one per SM,
@@ -330,7 +341,8 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const f
     return KD_ERR_CUDA;
   const int groups = resident_groups(dev);
   ProbArgs a{};
-  a.raster = forward_raster(ceil_div(N, GeoP::TILE_M), ceil_div(V, BN), groups);
+  a.raster = forward_raster(ceil_div(N, GeoP::TILE_M), ceil_div(V, BN), groups, GeoP::TILE_M * d * 2,
+                            device_l2_bytes(dev));
   a.num_kb = (int)ceil_div(d, BK);
   EpiFwd::Params ep{};
   ep.N = (int)N;
@@ -443,7 +455,7 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     a45.prob[1].raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
     a45.prob[1].num_kb = (int)ceil_div(Cc, BK);
     a45.prob[1].b_k0 = (int)c0;
-    balance_second_problem(a45, groups);
+    plan_second_problem(a45, groups);
     EpiDh::Params e4{};
     e4.row0 = (int)c0;
     EpiDw::Params e5{};

@@ -35,13 +35,14 @@ int main() {
   int cases = 0;
   for (long N : Ns)
     for (long V : Vs)
-      for (int g : grids) {
-        Raster r = forward_raster(ceil_div64(N, 128), ceil_div64(V, 256), g);
-        if (r.splits > kMaxSplits) { printf("FAIL splits %d\n", r.splits); return 1; }
-        if (r.group_m < 1) { printf("FAIL group_m\n"); return 1; }
-        if (!check(r, "fwd", N, V, g)) return 1;
-        ++cases;
-      }
+      for (int g : grids)
+        for (long d : ds) {
+          Raster r = forward_raster(ceil_div64(N, 128), ceil_div64(V, 256), g, 256 * d * 2, 126l << 20);
+          if (r.splits > kMaxSplits) { printf("FAIL splits %d\n", r.splits); return 1; }
+          if (r.group_m < 1 || r.group_m > r.m_tiles) { printf("FAIL group_m\n"); return 1; }
+          if (!check(r, "fwd", N, V, g)) return 1;
+          ++cases;
+        }
   for (long C : chunks)
     for (long V : Vs)
       for (long d : ds) {
@@ -50,30 +51,41 @@ int main() {
         if (!check(tile_raster(ceil_div64(V, 128), ceil_div64(d, 256), false), "dw", C, V, d)) return 1;
         cases += 3;
       }
-  // joint launches: every problem-1 unit in exactly one contiguous range,
-  // and no group's total more than one problem-1 unit above the ideal
+  // joint launches: every problem-1 unit dealt exactly once; when there are
+  // enough of them to even out the groups, no group's K blocks differ from
+  // another's by more than 1.5 problem-1 units
   const long U0s[] = {0, 1, 16, 32, 192, 400};
   const long k0s[] = {1, 45, 501, 3142};
   const long U1s[] = {0, 1, 12, 9432, 6012};
   const long k1s[] = {1, 16, 64};
+  std::vector<int> seen;
   for (long U0 : U0s)
     for (long k0 : k0s)
       for (long U1 : U1s)
         for (long k1 : k1s)
           for (int g : {1, 7, 74, 148}) {
-            int starts[257];
-            balance_ranges(U0, k0, U1, k1, g, starts);
-            if (starts[0] != 0 || starts[g] != U1) { printf("FAIL joint total\n"); return 1; }
-            double ideal = (double)(U0 * k0 + U1 * k1) / g;
-            long worst0 = ((U0 + g - 1) / g) * k0;
+            const JointPlan p = joint_plan(U0, k0, U1, k1, g);
+            seen.assign((size_t)U1, 0);
+            long lo = -1, hi = -1;
             for (int i = 0; i < g; ++i) {
-              if (starts[i + 1] < starts[i]) { printf("FAIL joint order\n"); return 1; }
-              long n0 = i < U0 ? (U0 - i + g - 1) / g : 0;
-              double tot = (double)(n0 * k0 + (long)(starts[i + 1] - starts[i]) * k1);
-              if (tot > ideal + k1 + 1e-6 && tot > (double)(n0 * k0) + 1e-6 && (double)worst0 < ideal) {
-                printf("FAIL joint balance U0 %ld k0 %ld U1 %ld k1 %ld g %d: %f vs %f\n", U0, k0, U1, k1, g, tot, ideal);
-                return 1;
+              const int n = joint_count(p, U1, g, i);
+              for (int j = 0; j < n; ++j) {
+                const int u = joint_unit(p, g, i, j);
+                if (u < 0 || u >= U1) { printf("FAIL joint unit %d of %ld\n", u, U1); return 1; }
+                ++seen[(size_t)u];
               }
+              const long n0 = i < U0 ? (U0 - i + g - 1) / g : 0;
+              const long tot = n0 * k0 + (long)n * k1;
+              lo = lo < 0 || tot < lo ? tot : lo;
+              hi = tot > hi ? tot : hi;
+            }
+            for (long u = 0; u < U1; ++u)
+              if (seen[(size_t)u] != 1) { printf("FAIL joint seen %d\n", seen[(size_t)u]); return 1; }
+            const long r = U0 % g;
+            const bool enough = r == 0 || (long)p.wb == (k0 + k1 / 2) / k1;
+            if (enough && U1 >= p.p2 + g && 2 * (hi - lo) > 3 * k1) {
+              printf("FAIL joint balance U0 %ld k0 %ld U1 %ld k1 %ld g %d: %ld..%ld\n", U0, k0, U1, k1, g, lo, hi);
+              return 1;
             }
             ++cases;
           }
