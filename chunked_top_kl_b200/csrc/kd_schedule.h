@@ -18,10 +18,10 @@ constexpr int kMaxSplits = 16;   // column ranges per band in the forward pass
 KD_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct Raster {
-  int m_tiles;          // 128-row bands
+  int m_tiles;          // row bands (one tile high)
   int n_tiles;          // 256-column tiles
   int splits;           // column ranges per band
-  int tiles_per_split;  // tiles in one range (the last may be shorter)
+  int tiles_per_split;  // tiles in the longest range
   int group_m;          // bands interleaved within one group of units
   int num_units;        // m_tiles * splits
 };
@@ -30,7 +30,8 @@ struct Raster {
 // Consecutive units (which run at the same time on different SMs) walk the
 // bands of a group fastest, then the ranges, then the groups; so the SMs of
 // one wave share column tiles (L2 reuse of the B operand) across group_m
-// bands while each band's A tile is shared across the ranges.
+// bands while each band's A tile is shared across the ranges.  Range lengths
+// differ by at most one tile, so units of one wave stay in step.
 KD_HD void decode_unit(const Raster& r, int u, int& m, int& split, int& n0, int& n1) {
   const int per_group = r.group_m * r.splits;
   const int g = u / per_group;
@@ -39,8 +40,10 @@ KD_HD void decode_unit(const Raster& r, int u, int& m, int& split, int& n0, int&
   const int rr = u - g * per_group;
   m = gm0 + rr % gsz;
   split = rr / gsz;
-  n0 = split * r.tiles_per_split;
-  n1 = (n0 + r.tiles_per_split < r.n_tiles) ? (n0 + r.tiles_per_split) : r.n_tiles;
+  const int base = r.n_tiles / r.splits;
+  const int extra = r.n_tiles - base * r.splits;
+  n0 = split * base + (split < extra ? split : extra);
+  n1 = n0 + base + (split < extra ? 1 : 0);
 }
 
 // One tile per unit; bands fastest (group_m = all bands) or column tiles
@@ -58,7 +61,7 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
 
 // Forward pass: a unit is a band and a range of vocabulary tiles whose
 // running log-sum-exp one CTA carries.  Picks the number of ranges
-// (<= kMaxSplits) minimising waves x tiles-per-unit on `grid` CTAs; every
+// (<= kMaxSplits) minimising waves x longest range on `grid` CTAs; every
 // range is non-empty.
 //
 // The B operand (the vocabulary rows) is the large one, so a wave should
@@ -71,16 +74,14 @@ inline Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid, int64_t
   int best_s = 1;
   int64_t best_cost = INT64_MAX;
   for (int s = 1; s <= kMaxSplits && s <= n_tiles; ++s) {
-    const int64_t tps = ceil_div64(n_tiles, s);
-    const int64_t se = ceil_div64(n_tiles, tps);
-    const int64_t cost = ceil_div64(m_tiles * se, grid) * tps;
-    if (cost < best_cost) { best_cost = cost; best_s = (int)se; }
+    const int64_t cost = ceil_div64(m_tiles * s, grid) * ceil_div64(n_tiles, s);
+    if (cost < best_cost) { best_cost = cost; best_s = s; }
   }
   Raster r;
   r.m_tiles = (int)m_tiles;
   r.n_tiles = (int)n_tiles;
+  r.splits = best_s;
   r.tiles_per_split = (int)ceil_div64(n_tiles, best_s);
-  r.splits = (int)ceil_div64(n_tiles, r.tiles_per_split);
   int64_t gm = grid / 2;
   if (band_bytes > 0 && l2_budget > 0) {
     const int64_t cap = l2_budget / 2 / band_bytes;
