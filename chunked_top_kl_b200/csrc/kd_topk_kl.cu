@@ -446,11 +446,12 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
       return KD_ERR_CUDA;
 
     // One launch for both gradient products of the chunk:
-    //   problem 0: dH[chunk] = dZ W      (few long tiles, K = V)
+    //   problem 0: dH[chunk] = dZ W      (few long tiles, K = V; a band's column
+    //              tiles side by side, so each dZ band is fetched once per wave)
     //   problem 1: dW (+)= dZ^T H[chunk] (many short tiles, K = chunk)
     GemmArgs a45{};
     a45.status = status;
-    a45.prob[0].raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), true);
+    a45.prob[0].raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), false);
     a45.prob[0].num_kb = (int)ceil_div(V, BK);
     a45.prob[1].raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
     a45.prob[1].num_kb = (int)ceil_div(Cc, BK);
