@@ -47,6 +47,20 @@ T^2 factor); duplicate teacher indices add their probabilities at that
 column; an index outside ``[0, V)`` is an error; masked tokens still get an
 lse; a teacher logit of ``-inf`` gives ``p = 0`` and contributes nothing.
 
+Variants (not on the pages; options of the library, defaults off):
+  * An index of ``-1`` marks an empty teacher slot (a cache with fewer than
+    K entries for some tokens).  Empty slots take no part in step 3's
+    softmax, so ``p`` is renormalised over the filled slots.  A token with no
+    filled slot has an empty teacher distribution: ``P_n = sum_k p_k = 0``,
+    ``term_n = 0`` and, since ``d term_n / dz = P_n softmax(z) - scatter(p)``,
+    a zero dZ row.  Its mask still counts in ``sum m``.
+  * ``student_T``: the usual distillation temperature, applied to the
+    student too: steps 2 and 4 use ``z / T`` in place of ``z`` (``lse`` is
+    then ``logsumexp(z / T)``) and ``term_n`` is multiplied by ``T^2``, so
+    step 7 becomes ``dZ = c_n T (softmax(z / T) - scatter(p))``.
+  * A bf16 teacher cache needs nothing here: the oracle takes the logits'
+    values, whatever type held them.
+
 Tokens are processed in row blocks only to bound memory; every quantity
 above is per token except the sums over n in steps 5 and 9, which are
 accumulated block by block in fp64.  Matrix products use numpy's fp64
@@ -95,13 +109,22 @@ def _rows_per_block(V: int) -> int:
     return max(1, _BLOCK_ELEMS // max(1, V))
 
 
-def teacher_distribution(logit: np.ndarray, T: float):
+def teacher_distribution(logit: np.ndarray, T: float, filled: Optional[np.ndarray] = None):
     """Step 3: ``p`` and ``log p`` of the temperature softmax over each row's K
-    cached teacher logits.  Rows of ``logit`` are tokens."""
+    cached teacher logits.  Rows of ``logit`` are tokens.  ``filled`` (bool,
+    same shape) marks the slots that hold an entry; the others get ``p = 0``
+    and take no part in the normalisation.  A row without a finite filled
+    logit gets ``p = 0`` throughout."""
     t = as_f64(logit) / float(T)
-    tmax = np.max(t, axis=1, keepdims=True)
-    lse_t = tmax + np.log(np.sum(np.exp(t - tmax), axis=1, keepdims=True))
-    logp = t - lse_t
+    if filled is not None:
+        t = np.where(filled, t, -np.inf)
+    tmax = np.max(t, axis=1, keepdims=True) if t.shape[1] else np.full((t.shape[0], 1), -np.inf)
+    empty = ~np.isfinite(tmax[:, 0])
+    tmax = np.where(np.isfinite(tmax), tmax, 0.0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lse_t = tmax + np.log(np.sum(np.exp(t - tmax), axis=1, keepdims=True))
+        logp = t - lse_t
+    logp[empty] = -np.inf
     p = np.exp(logp)
     return p, logp
 
@@ -112,9 +135,19 @@ def student_lse(z: np.ndarray) -> np.ndarray:
     return (zmax + np.log(np.sum(np.exp(z - zmax), axis=1, keepdims=True)))[:, 0]
 
 
+EMPTY_SLOT = -1   # teacher index of an empty cache slot
+
+
 def _check_idx(idx: np.ndarray, V: int) -> None:
-    if idx.size and (idx.min() < 0 or idx.max() >= V):
+    if idx.size and (idx.min() < EMPTY_SLOT or idx.max() >= V or np.any((idx < 0) & (idx != EMPTY_SLOT))):
         raise ValueError("teacher index outside [0, V)")
+
+
+def _slots(idx: np.ndarray):
+    """Filled-slot mask, and indices with empty slots pointed at column 0
+    (their p is 0, so they add nothing there)."""
+    filled = idx != EMPTY_SLOT
+    return filled, np.where(filled, idx, 0)
 
 
 def _token_terms(z: np.ndarray, lse: np.ndarray, idx: np.ndarray,
@@ -128,8 +161,9 @@ def _token_terms(z: np.ndarray, lse: np.ndarray, idx: np.ndarray,
 
 def _dz_block(z: np.ndarray, lse: np.ndarray, idx: np.ndarray, p: np.ndarray,
               c: np.ndarray) -> np.ndarray:
-    """Step 7 for a block of tokens."""
-    q = np.exp(z - lse[:, None])
+    """Step 7 for a block of tokens: ``c_n (P_n softmax(z) - scatter(p))`` with
+    ``P_n = sum_k p_k`` (1, or 0 for a token without teacher entries)."""
+    q = np.exp(z - lse[:, None]) * np.sum(p, axis=1, keepdims=True)
     scat = np.zeros_like(q)
     rows = np.repeat(np.arange(z.shape[0]), idx.shape[1])
     np.add.at(scat, (rows, idx.reshape(-1)), p.reshape(-1))
@@ -137,20 +171,24 @@ def _dz_block(z: np.ndarray, lse: np.ndarray, idx: np.ndarray, p: np.ndarray,
 
 
 def kd_topk_kl(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0,
-               grad: float = 1.0, backward: bool = True) -> Dict[str, object]:
+               grad: float = 1.0, backward: bool = True, student_T: bool = False) -> Dict[str, object]:
     """Steps 1-9 for all tokens.  Returns ``loss`` (float), ``lse`` [N],
     ``term`` [N], ``sum_mask`` and, if ``backward``, ``dH`` [N,d] and
-    ``dW`` [V,d]; all fp64."""
+    ``dW`` [V,d]; all fp64.  ``student_T`` selects the variant with the
+    student at temperature T and the T^2 factor."""
     Hf = as_f64(H)
     Wf = as_f64(W)
     idx = _as_i64(topk_idx)
     N, d = Hf.shape
     V = Wf.shape[0]
     _check_idx(idx, V)
+    filled, idx = _slots(idx)
     m = np.ones(N) if mask is None else as_f64(mask)
-    p, logp = teacher_distribution(topk_logit, T)
+    p, logp = teacher_distribution(topk_logit, T, filled)
     sum_mask = float(np.sum(m))
     c = (grad * m / sum_mask) if sum_mask != 0.0 else np.zeros(N)
+    zs = 1.0 / float(T) if student_T else 1.0            # student logits used: z * zs
+    tfac = float(T) ** 2 if student_T else 1.0           # factor on term_n
 
     lse = np.empty(N)
     term = np.empty(N)
@@ -159,11 +197,11 @@ def kd_topk_kl(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0,
     B = _rows_per_block(V)
     for s in range(0, N, B):
         e = min(N, s + B)
-        z = Hf[s:e] @ Wf.T                                   # step 1
+        z = (Hf[s:e] @ Wf.T) * zs                            # step 1
         lse[s:e] = student_lse(z)                            # step 2
-        term[s:e] = _token_terms(z, lse[s:e], idx[s:e], p[s:e], logp[s:e])  # step 4
+        term[s:e] = tfac * _token_terms(z, lse[s:e], idx[s:e], p[s:e], logp[s:e])  # step 4
         if backward:
-            dz = _dz_block(z, lse[s:e], idx[s:e], p[s:e], c[s:e])           # step 7
+            dz = _dz_block(z, lse[s:e], idx[s:e], p[s:e], c[s:e] * (tfac * zs))  # step 7
             dH[s:e] = dz @ Wf                                # step 8
             dW += dz.T @ Hf[s:e]                             # step 9
     loss = float(np.sum(m * term) / sum_mask) if sum_mask != 0.0 else 0.0   # step 5
@@ -174,15 +212,16 @@ def kd_topk_kl(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0,
     return out
 
 
-def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0):
+def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, student_T: bool = False):
     """Steps 1-5: ``(loss, lse)``."""
-    r = kd_topk_kl(H, W, topk_idx, topk_logit, mask, T, backward=False)
+    r = kd_topk_kl(H, W, topk_idx, topk_logit, mask, T, backward=False, student_T=student_T)
     return r["loss"], r["lse"]
 
 
-def backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, grad: float = 1.0):
+def backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, grad: float = 1.0,
+             student_T: bool = False):
     """Steps 6-9: ``(dH, dW)``."""
-    r = kd_topk_kl(H, W, topk_idx, topk_logit, mask, T, grad=grad)
+    r = kd_topk_kl(H, W, topk_idx, topk_logit, mask, T, grad=grad, student_T=student_T)
     return r["dH"], r["dW"]
 
 
@@ -203,7 +242,8 @@ def term_rows(H, W, topk_idx, topk_logit, rows: Sequence[int], T: float = 1.0):
     Wf = as_f64(W)
     idx = _as_i64(topk_idx)[rows]
     _check_idx(idx, Wf.shape[0])
-    p, logp = teacher_distribution(as_f64(topk_logit)[rows], T)
+    filled, idx = _slots(idx)
+    p, logp = teacher_distribution(as_f64(topk_logit)[rows], T, filled)
     z = Hf @ Wf.T
     lse = student_lse(z)
     return lse, _token_terms(z, lse, idx, p, logp)
@@ -220,7 +260,8 @@ def dH_rows(H, W, topk_idx, topk_logit, mask, rows: Sequence[int], T: float = 1.
     m_all = np.ones(as_f64(topk_logit).shape[0]) if mask is None else as_f64(mask)
     sum_mask = float(np.sum(m_all))
     c = grad * m_all[rows] / sum_mask if sum_mask != 0.0 else np.zeros(len(rows))
-    p, _ = teacher_distribution(as_f64(topk_logit)[rows], T)
+    filled, idx = _slots(idx)
+    p, _ = teacher_distribution(as_f64(topk_logit)[rows], T, filled)
     z = Hf @ Wf.T
     lse = student_lse(z)
     return _dz_block(z, lse, idx, p, c) @ Wf
@@ -240,14 +281,16 @@ def dW_rows(H, W, topk_idx, topk_logit, mask, lse: np.ndarray, vrows: Sequence[i
     m = np.ones(N) if mask is None else as_f64(mask)
     sum_mask = float(np.sum(m))
     c = grad * m / sum_mask if sum_mask != 0.0 else np.zeros(N)
-    p, _ = teacher_distribution(topk_logit, T)
+    filled, idx = _slots(idx)
+    p, _ = teacher_distribution(topk_logit, T, filled)
+    psum = np.sum(p, axis=1)
     lse = np.asarray(lse, dtype=np.float64)
     out = np.zeros((len(vrows), Hf.shape[1]))
     B = _rows_per_block(len(vrows))
     for s in range(0, N, B):
         e = min(N, s + B)
         z = Hf[s:e] @ Wv.T                                   # z[n, vrows]
-        q = np.exp(z - lse[s:e, None])
+        q = np.exp(z - lse[s:e, None]) * psum[s:e, None]
         scat = np.zeros_like(q)
         for j, v in enumerate(vrows):
             scat[:, j] = np.sum(np.where(idx[s:e] == v, p[s:e], 0.0), axis=1)

@@ -15,7 +15,10 @@ and show that every planted mistake is caught.
 * teacher logits equal to student logits over the whole vocabulary give a
   zero loss and zero gradients;
 * KL >= 0; invariances; central finite differences;
-* hand-derived worked examples under ``tests/golden/``.
+* hand-derived worked examples under ``tests/golden/``;
+* the library's variants (empty slots marked by index -1, the student at
+  temperature T with the T^2 factor): dense torch references with autograd,
+  compaction of empty slots, finite differences.
 """
 
 from __future__ import annotations
@@ -67,8 +70,31 @@ def _torch_dense(H, W, idx, logit, mask, T, grad=1.0):
     return (loss.item(), torch.logsumexp(z, 1).detach().numpy(), H.grad.numpy(), W.grad.numpy())
 
 
-def _run(orc, H, W, idx, logit, mask, T, grad=1.0):
-    return orc.kd_topk_kl(H.numpy(), W.numpy(), idx.numpy(), logit.numpy(), mask.numpy(), T, grad=grad)
+def _run(orc, H, W, idx, logit, mask, T, grad=1.0, **kw):
+    return orc.kd_topk_kl(H.numpy(), W.numpy(), idx.numpy(), logit.numpy(), mask.numpy(), T, grad=grad, **kw)
+
+
+def _torch_dense_variant(H, W, idx, logit, mask, T, grad=1.0, student_T=False):
+    """Dense reference of the library's variants: slots with index -1 hold no
+    entry (the teacher softmax runs over the filled slots only; a row with
+    none has an all-zero teacher grid), and with ``student_T`` the student
+    log-softmax is taken of z / T and the loss multiplied by T^2."""
+    H = H.clone().requires_grad_(True)
+    W = W.clone().requires_grad_(True)
+    z = H @ W.T
+    logq = torch.log_softmax(z / T if student_T else z, dim=1)
+    filled = idx != -1
+    t = torch.where(filled, logit / T, torch.full_like(logit, -math.inf))
+    any_filled = filled.any(dim=1, keepdim=True)
+    p = torch.where(any_filled, torch.softmax(torch.where(any_filled, t, torch.zeros_like(t)), dim=1),
+                    torch.zeros_like(t))
+    p = torch.where(filled, p, torch.zeros_like(p))
+    P = torch.zeros_like(z).scatter_add(1, torch.where(filled, idx, torch.zeros_like(idx)), p)
+    kl = F.kl_div(logq, P, reduction="none").sum(dim=1)
+    loss = (T * T if student_T else 1.0) * (mask * kl).sum() / mask.sum()
+    (grad * loss).backward()
+    lse = torch.logsumexp(z / T if student_T else z, 1)
+    return (loss.item(), lse.detach().numpy(), H.grad.numpy(), W.grad.numpy())
 
 
 def _close(a, b, tol, what):
@@ -210,8 +236,82 @@ def pin_golden(orc):
         _close(r["dW"], [[eval(e, env) for e in row] for row in ex["dW"]], 1e-14, case["name"] + " dW")
 
 
+def _empty_slots(idx, seed, frac=0.4, empty_row=True):
+    g = torch.Generator().manual_seed(1000 + seed)
+    idx = idx.clone()
+    idx[torch.rand(idx.shape, generator=g) < frac] = -1
+    if empty_row and idx.shape[0] > 2:
+        idx[2] = -1
+    return idx
+
+
+def pin_empty_slots_dense(orc):
+    # variant: index -1 marks an empty slot; a row without entries adds nothing
+    for seed, kw in [(30, {}), (31, {"T": 2.0, "K": 6}), (32, {"V": 40, "K": 12, "N": 9, "masked": False})]:
+        H, W, idx, logit, mask, T = _rand_case(seed, **kw)
+        idx = _empty_slots(idx, seed)
+        r = _run(orc, H, W, idx, logit, mask, T, grad=1.3)
+        loss, lse, dH, dW = _torch_dense_variant(H, W, idx, logit, mask, T, grad=1.3)
+        _close(r["loss"], loss, 1e-12, f"loss seed {seed}")
+        _close(r["lse"], lse, 1e-12, f"lse seed {seed}")
+        _close(r["dH"], dH, 1e-12, f"dH seed {seed}")
+        _close(r["dW"], dW, 1e-12, f"dW seed {seed}")
+        assert r["term"][2] == 0.0 and np.all(r["dH"][2] == 0.0)
+
+
+def pin_empty_slots_compaction(orc):
+    # every row with the same number of filled slots == the cache without them
+    H, W, idx, logit, mask, T = _rand_case(33, N=6, V=15, K=7, T=1.4)
+    g = torch.Generator().manual_seed(33)
+    keep = torch.stack([torch.randperm(7, generator=g)[:4].sort().values for _ in range(6)])
+    padded = torch.full_like(idx, -1)
+    padded.scatter_(1, keep, idx.gather(1, keep))
+    r = _run(orc, H, W, padded, logit, mask, T, grad=0.8)
+    c = _run(orc, H, W, idx.gather(1, keep), logit.gather(1, keep), mask, T, grad=0.8)
+    for k in ("loss", "lse", "term", "dH", "dW"):
+        _close(r[k], c[k], 1e-13, "compaction " + k)
+
+
+def pin_student_temperature_dense(orc):
+    # variant: the student at temperature T too, loss times T^2
+    for seed, kw, empty in [(34, {"T": 2.0}, False), (35, {"T": 0.5, "K": 6}, False),
+                            (36, {"T": 3.0, "V": 30, "K": 8, "N": 8}, True)]:
+        H, W, idx, logit, mask, T = _rand_case(seed, **kw)
+        if empty:
+            idx = _empty_slots(idx, seed)
+        r = _run(orc, H, W, idx, logit, mask, T, grad=0.9, student_T=True)
+        loss, lse, dH, dW = _torch_dense_variant(H, W, idx, logit, mask, T, grad=0.9, student_T=True)
+        _close(r["loss"], loss, 1e-12, f"loss seed {seed}")
+        _close(r["lse"], lse, 1e-12, f"lse seed {seed}")
+        _close(r["dH"], dH, 1e-12, f"dH seed {seed}")
+        _close(r["dW"], dW, 1e-12, f"dW seed {seed}")
+
+
+def pin_student_temperature_fd(orc):
+    # central finite differences of the variant's loss
+    H, W, idx, logit, mask, T = _rand_case(37, N=3, d=4, V=9, K=3, T=1.7)
+    Hn, Wn, In, Ln, Mn = H.numpy(), W.numpy(), idx.numpy(), logit.numpy(), mask.numpy()
+    r = orc.kd_topk_kl(Hn, Wn, In, Ln, Mn, T, grad=1.0, student_T=True)
+    L = lambda a, b: orc.kd_topk_kl(a, b, In, Ln, Mn, T, backward=False, student_T=True)["loss"]
+    h = 1e-6
+    for (i, j) in [(0, 0), (1, 2), (2, 3)]:
+        Hp, Hm = Hn.copy(), Hn.copy()
+        Hp[i, j] += h
+        Hm[i, j] -= h
+        fd = (L(Hp, Wn) - L(Hm, Wn)) / (2 * h)
+        assert abs(fd - r["dH"][i, j]) <= 1e-6 * max(1e-3, abs(fd)) + 1e-9, ("dH", i, j, fd, r["dH"][i, j])
+    for (v, j) in [(0, 1), (4, 0), (8, 3)]:
+        Wp, Wm = Wn.copy(), Wn.copy()
+        Wp[v, j] += h
+        Wm[v, j] -= h
+        fd = (L(Hn, Wp) - L(Hn, Wm)) / (2 * h)
+        assert abs(fd - r["dW"][v, j]) <= 1e-6 * max(1e-3, abs(fd)) + 1e-9, ("dW", v, j, fd, r["dW"][v, j])
+
+
 PINS = [pin_bruteforce_dense, pin_duplicate_gradient, pin_cross_entropy_k1, pin_w_zero,
-        pin_equal_teacher, pin_kl_nonneg, pin_invariances, pin_finite_differences, pin_golden]
+        pin_equal_teacher, pin_kl_nonneg, pin_invariances, pin_finite_differences, pin_golden,
+        pin_empty_slots_dense, pin_empty_slots_compaction, pin_student_temperature_dense,
+        pin_student_temperature_fd]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -234,7 +334,7 @@ def test_bad_index_rejected():
     idx[0, 0] = W.shape[0]
     with pytest.raises(ValueError):
         _run(ORACLE, H, W, idx, logit, mask, T)
-    idx[0, 0] = -1
+    idx[0, 0] = -2          # -1 is an empty slot, any other negative index an error
     with pytest.raises(ValueError):
         _run(ORACLE, H, W, idx, logit, mask, T)
 
@@ -279,6 +379,12 @@ MUTANTS = {
     "mask_not_normalised": ("loss = float(np.sum(m * term) / sum_mask)", "loss = float(np.sum(m * term) / len(m))"),
     "dW_uses_wrong_operand": ("dW += dz.T @ Hf[s:e]", "dW += dz.T @ Hf[s:e] * 0.5"),
     "dH_dropped_term": ("dH[s:e] = dz @ Wf", "dH[s:e] = (dz * (dz > 0)) @ Wf"),
+    "empty_slot_in_softmax": ("t = np.where(filled, t, -np.inf)", "t = np.where(filled, t, t)"),
+    "empty_row_keeps_softmax": ("q = np.exp(z - lse[:, None]) * np.sum(p, axis=1, keepdims=True)",
+                                "q = np.exp(z - lse[:, None])"),
+    "student_T_not_squared": ("tfac = float(T) ** 2 if student_T else 1.0", "tfac = float(T) if student_T else 1.0"),
+    "student_T_student_unscaled": ("zs = 1.0 / float(T) if student_T else 1.0", "zs = 1.0"),
+    "student_T_grad_scale": ("c[s:e] * (tfac * zs)", "c[s:e] * tfac"),
 }
 
 
