@@ -29,7 +29,24 @@ EXPORTS = (
     "kd_topk_kl_forward_noalloc",
     "kd_topk_kl_backward_profiled",
     "kd_topk_kl_forward_backward",
+    "kd_topk_kl_forward_ex",
+    "kd_topk_kl_backward_ex",
+    "kd_topk_kl_forward_backward_ex",
 )
+
+
+class KDOptions(ctypes.Structure):
+    """kd_topk_kl_options (see the C header)."""
+    _fields_ = [("logit_bf16", ctypes.c_int32), ("student_temperature", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
+
+
+def make_options(logit_bf16: bool = False, student_temperature: bool = False) -> KDOptions:
+    o = KDOptions()
+    o.logit_bf16 = int(bool(logit_bf16))
+    o.student_temperature = int(bool(student_temperature))
+    return o
+
 
 _lib = None
 
@@ -62,6 +79,16 @@ def load() -> ctypes.CDLL:
         lib.kd_topk_kl_forward_backward.restype = i32
         lib.kd_topk_kl_forward_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, p, p, p]
         lib.kd_topk_kl_forward_noalloc.restype = i32
+        opt = ctypes.POINTER(KDOptions)
+        evp = ctypes.POINTER(ctypes.c_void_p)
+        lib.kd_topk_kl_forward_ex.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p, sz, p, opt]
+        lib.kd_topk_kl_forward_ex.restype = i32
+        lib.kd_topk_kl_backward_ex.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p, p, i32,
+                                               p, sz, p, evp, i64, opt]
+        lib.kd_topk_kl_backward_ex.restype = i32
+        lib.kd_topk_kl_forward_backward_ex.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p,
+                                                       p, p, i32, p, sz, p, evp, i64, opt]
+        lib.kd_topk_kl_forward_backward_ex.restype = i32
         _lib = lib
     return _lib
 
@@ -131,3 +158,38 @@ def kd_topk_kl_forward_noalloc(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, 
     callers that cannot allocate device memory (see the C header)."""
     return int(load().kd_topk_kl_forward_noalloc(H, W, topk_idx, topk_logit, mask, N, d, V, K, T,
                                                  loss, lse, stream))
+
+
+def _events(events):
+    if events:
+        return (ctypes.c_void_p * len(events))(*events), len(events)
+    return None, 0
+
+
+def _opt(options):
+    return None if options is None else ctypes.byref(options)
+
+
+def kd_topk_kl_forward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, loss, lse,
+                          workspace, workspace_bytes, stream, options=None) -> int:
+    return int(load().kd_topk_kl_forward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk,
+                                            loss, lse, workspace, workspace_bytes, stream, _opt(options)))
+
+
+def kd_topk_kl_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse, grad_loss,
+                           dH, dW, accumulate_dW, workspace, workspace_bytes, stream, events=None,
+                           options=None) -> int:
+    arr, n = _events(events)
+    return int(load().kd_topk_kl_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk,
+                                             lse, grad_loss, dH, dW, int(accumulate_dW), workspace,
+                                             workspace_bytes, stream, arr, n, _opt(options)))
+
+
+def kd_topk_kl_forward_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, loss, lse,
+                                   grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes, stream,
+                                   events=None, options=None) -> int:
+    arr, n = _events(events)
+    return int(load().kd_topk_kl_forward_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T,
+                                                     chunk, loss, lse, grad_loss, dH, dW,
+                                                     int(accumulate_dW), workspace, workspace_bytes,
+                                                     stream, arr, n, _opt(options)))

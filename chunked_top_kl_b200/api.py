@@ -20,8 +20,8 @@ def _check_inputs(H, W, topk_idx, topk_logit, mask):
         raise ValueError("kd_topk_kl: all inputs must be CUDA tensors")
     if H.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
         raise TypeError("kd_topk_kl: H and W must be bfloat16")
-    if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
-        raise TypeError("kd_topk_kl: topk_idx must be int32 and topk_logit float32")
+    if topk_idx.dtype != torch.int32 or topk_logit.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("kd_topk_kl: topk_idx must be int32 and topk_logit float32 or bfloat16")
     if mask is not None and (mask.dtype != torch.float32 or not mask.is_cuda):
         raise TypeError("kd_topk_kl: mask must be a float32 CUDA tensor")
     for t in (H, W, topk_idx, topk_logit) + ((mask,) if mask is not None else ()):
@@ -53,9 +53,21 @@ def _raise(st: int, where: str):
         raise _abi.KDError(st, where)
 
 
+def _options(topk_logit, student_temperature: bool):
+    """kd_topk_kl_options for these inputs, or None for the default loss
+    (fp32 logits, T on the teacher only): the plain entry points then run."""
+    bf16 = topk_logit.dtype == torch.bfloat16
+    if not bf16 and not student_temperature:
+        return None
+    return _abi.make_options(logit_bf16=bf16, student_temperature=student_temperature)
+
+
 def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
-            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Returns (loss [] fp32, lse [N] fp32)."""
+            workspace: Optional[torch.Tensor] = None,
+            student_temperature: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Returns (loss [] fp32, lse [N] fp32).  ``topk_logit`` may be fp32 or
+    bf16; ``student_temperature`` selects the variant with the student
+    logits divided by T too and the loss multiplied by T^2."""
     N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
     dev = H.device
     if workspace is None:
@@ -63,10 +75,17 @@ def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 
     loss = torch.empty((), dtype=torch.float32, device=dev)
     lse = torch.empty(N, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    st = _abi.kd_topk_kl_forward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
-                                 N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
-                                 _ptr(workspace), workspace.numel(), stream)
-    _raise(st, "kd_topk_kl_forward")
+    opt = _options(topk_logit, student_temperature)
+    if opt is None:
+        st = _abi.kd_topk_kl_forward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                     N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
+                                     _ptr(workspace), workspace.numel(), stream)
+        _raise(st, "kd_topk_kl_forward")
+    else:
+        st = _abi.kd_topk_kl_forward_ex(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                        N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
+                                        _ptr(workspace), workspace.numel(), stream, opt)
+        _raise(st, "kd_topk_kl_forward_ex")
     return loss, lse
 
 
@@ -78,10 +97,12 @@ def backward_launches(N: int, chunk: int) -> int:
 def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.Tensor,
              grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
              accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
-             dH: Optional[torch.Tensor] = None, events=None) -> Tuple[torch.Tensor, torch.Tensor]:
+             dH: Optional[torch.Tensor] = None, events=None,
+             student_temperature: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Returns (dH [N,d] bf16, dW [V,d] fp32).  With ``events`` (a list of
     backward_launches(N, chunk) + 1 created torch.cuda.Event objects) the
-    library records them around each of its kernel launches."""
+    library records them around each of its kernel launches.
+    ``student_temperature`` must match the forward call that made ``lse``."""
     N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
     dev = H.device
     if workspace is None:
@@ -94,7 +115,15 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
     if grad_loss is not None:
         grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    if events is None:
+    opt = _options(topk_logit, student_temperature)
+    if opt is not None:
+        st = _abi.kd_topk_kl_backward_ex(
+            _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
+            int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+            _ptr(workspace), workspace.numel(), stream,
+            None if events is None else [e.cuda_event for e in events], opt)
+        _raise(st, "kd_topk_kl_backward_ex")
+    elif events is None:
         st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
                                       N, d, V, K, float(T), int(chunk), _ptr(lse), _ptr(grad_loss),
                                       _ptr(dH), _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
@@ -117,7 +146,7 @@ def forward_backward_launches(N: int, chunk: int) -> int:
 def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
                      grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
                      accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
-                     dH: Optional[torch.Tensor] = None, events=None):
+                     dH: Optional[torch.Tensor] = None, events=None, student_temperature: bool = False):
     """One call for a training step: returns (loss, lse, dH, dW)."""
     N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
     dev = H.device
@@ -133,12 +162,15 @@ def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chun
     if grad_loss is not None:
         grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    st = _abi.kd_topk_kl_forward_backward(
-        _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T), int(chunk),
-        _ptr(loss), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
-        _ptr(workspace), workspace.numel(), stream,
-        None if events is None else [e.cuda_event for e in events])
-    _raise(st, "kd_topk_kl_forward_backward")
+    evs = None if events is None else [e.cuda_event for e in events]
+    opt = _options(topk_logit, student_temperature)
+    args = (_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T), int(chunk),
+            _ptr(loss), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+            _ptr(workspace), workspace.numel(), stream)
+    if opt is None:
+        _raise(_abi.kd_topk_kl_forward_backward(*args, evs), "kd_topk_kl_forward_backward")
+    else:
+        _raise(_abi.kd_topk_kl_forward_backward_ex(*args, evs, opt), "kd_topk_kl_forward_backward_ex")
     return loss, lse, dH, dW
 
 
@@ -151,22 +183,24 @@ def check(workspace: torch.Tensor) -> Tuple[int, int]:
 
 class KDTopKKLFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, H, W, topk_idx, topk_logit, mask, T, chunk):
-        loss, lse = forward(H, W, topk_idx, topk_logit, mask, T, chunk)
+    def forward(ctx, H, W, topk_idx, topk_logit, mask, T, chunk, student_temperature=False):
+        loss, lse = forward(H, W, topk_idx, topk_logit, mask, T, chunk,
+                            student_temperature=student_temperature)
         ctx.save_for_backward(H, W, topk_idx, topk_logit, mask, lse)
-        ctx.T, ctx.chunk = T, chunk
+        ctx.T, ctx.chunk, ctx.student_temperature = T, chunk, student_temperature
         return loss
 
     @staticmethod
     def backward(ctx, grad):
         H, W, topk_idx, topk_logit, mask, lse = ctx.saved_tensors
         dH, dW = backward(H, W, topk_idx, topk_logit, mask, ctx.T, ctx.chunk, lse,
-                          grad_loss=grad.reshape(()))
-        return dH, dW.to(W.dtype), None, None, None, None, None
+                          grad_loss=grad.reshape(()), student_temperature=ctx.student_temperature)
+        return dH, dW.to(W.dtype), None, None, None, None, None, None
 
 
-def kd_topk_kl_loss(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096):
+def kd_topk_kl_loss(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
+                    student_temperature: bool = False):
     """Differentiable loss (autograd).  dW is accumulated in fp32 inside the
     library and cast to W's dtype for autograd; call ``backward`` directly to
     keep an fp32 gradient."""
-    return KDTopKKLFunction.apply(H, W, topk_idx, topk_logit, mask, T, chunk)
+    return KDTopKKLFunction.apply(H, W, topk_idx, topk_logit, mask, T, chunk, student_temperature)

@@ -446,11 +446,14 @@ __device__ __forceinline__ int lower_bound_row(const int32_t* row, int len, int 
 
 // Forward: running max / sum-exp over the unit's vocabulary columns and the
 // gathered sum of p * z at the teacher's columns; one (m, s, g) partial per
-// token per split.  Columns >= V are -inf.
+// token per split.  Columns >= V are -inf.  The sum is of exp((z - m) * zs)
+// (zs = 1, or 1 / T when the student is taken at temperature T), computed as
+// 2^(z * zl2 - m * zl2) with zl2 = zs log2(e).
 struct EpiFwd {
   static constexpr bool kStaging = false;
   struct Params {
     int N, V, Kp;
+    float zl2;
     const int32_t* tidx;
     const float* tp;
     float* part_m;
@@ -513,16 +516,24 @@ struct EpiFwd {
         for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
       const float mn = fmaxf(mrun, t[0]);
       if (mn == -INFINITY) continue;
-      const float mb = mn * kLog2e;
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      // packed fp32 pairs (FFMA2 / FADD2) halve the epilogue's FMA and add
+      // instructions, which compete with the MMA issue for the SM
+      const float zl2 = P.zl2;
+      const float mb = mn * zl2;
+      const float2 zl2v = make_float2(zl2, zl2), nmb = make_float2(-mb, -mb);
+      float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i = 0; i < 64; i += 4) {
-        a0 += ex2_approx(fmaf(v[i + 0], kLog2e, -mb));
-        a1 += ex2_approx(fmaf(v[i + 1], kLog2e, -mb));
-        a2 += ex2_approx(fmaf(v[i + 2], kLog2e, -mb));
-        a3 += ex2_approx(fmaf(v[i + 3], kLog2e, -mb));
+        float2 e01 = __ffma2_rn(make_float2(v[i + 0], v[i + 1]), zl2v, nmb);
+        float2 e23 = __ffma2_rn(make_float2(v[i + 2], v[i + 3]), zl2v, nmb);
+        e01.x = ex2_approx(e01.x);
+        e01.y = ex2_approx(e01.y);
+        e23.x = ex2_approx(e23.x);
+        e23.y = ex2_approx(e23.y);
+        a01 = __fadd2_rn(a01, e01);
+        a23 = __fadd2_rn(a23, e23);
       }
-      srun = srun * ex2_approx((mrun - mn) * kLog2e) + ((a0 + a1) + (a2 + a3));
+      srun = srun * ex2_approx((mrun - mn) * zl2) + ((a01.x + a01.y) + (a23.x + a23.y));
       mrun = mn;
     }
   }
@@ -542,18 +553,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Backward, per chunk: dZ = c_n (exp(z - lse_n) - p at the teacher's columns),
-// rounded to bf16 and stored for the chunk's tokens (row-major, ldz columns)
-// through shared memory and TMA (`out`: the chunk buffer, bf16, box
-// {64, 128}, 128-byte swizzle).  Columns in [V, ldz) and rows at or past the
-// chunk's end (up to the buffer's rows) are written as 0, so that a buffer
-// reused for a shorter last chunk holds no stale rows.
+// Backward, per chunk: dZ = c_n (exp(z zs - lse_n) - p at the teacher's
+// columns), rounded to bf16 and stored for the chunk's tokens (row-major,
+// ldz columns) through shared memory and TMA (`out`: the chunk buffer, bf16,
+// box {64, 128}, 128-byte swizzle).  zs = 1, or 1 / T for the
+// student-temperature variant, whose extra factor T on c_n comes in as gfac.
+// A token without teacher entries has a zero row.  Columns in [V, ldz) and
+// rows at or past the chunk's end (up to the buffer's rows) are written as 0,
+// so that a buffer reused for a shorter last chunk holds no stale rows.
 struct EpiDz {
   static constexpr bool kStaging = true;
   struct Params {
     int rows_valid;        // tokens in this chunk
     int row0;              // global token index of chunk row 0
     int V, ldz, Kp;
+    float zl2;             // zs log2(e)
+    float gfac;            // 1, or T
     const int32_t* tidx;
     const float* tp;
     const float* lse;
@@ -567,11 +582,11 @@ struct EpiDz {
                                        uint32_t taddr, EpiCtx& cx) {
     const bool valid = r < P.rows_valid;
     const int grow = P.row0 + r;
-    // c exp(z - lse) = 2^(z log2(e) - bias) with bias = lse log2(e) - log2(c):
-    // one FFMA and one ex2 per element.  c = 0 (masked token) and rows past
-    // the chunk give bias = +inf, hence exact zeros.
-    // A negative c (negative upstream gradient or mask weight) is applied
-    // as a sign flip of the packed bf16 pair.
+    // c exp(z zs - lse) = 2^(z zl2 - bias) with bias = lse log2(e) - log2(c):
+    // one FFMA and one ex2 per element.  c = 0 (masked token, token without
+    // teacher entries) and rows past the chunk give bias = +inf, hence exact
+    // zeros.  A negative c (negative upstream gradient or mask weight) is
+    // applied as a sign flip of the packed bf16 pair.
     float bias = INFINITY, c = 0.f;
     uint32_t sgn = 0u;
     const int32_t* trow = nullptr;
@@ -579,24 +594,30 @@ struct EpiDz {
     int cur = 0, nidx = kSentinel;
     float np = 0.f;
     if (valid) {
-      const float cs = (P.mask ? P.mask[grow] : 1.f) * (*P.cscale);
+      trow = P.tidx + (size_t)grow * P.Kp;
+      prow = P.tp + (size_t)grow * P.Kp;
+      const float cs = trow[0] == kSentinel ? 0.f : (P.mask ? P.mask[grow] : 1.f) * (*P.cscale) * P.gfac;
       c = fabsf(cs);
       sgn = cs < 0.f ? 0x80008000u : 0u;
       bias = P.lse[grow] * kLog2e - log2f(c);
-      trow = P.tidx + (size_t)grow * P.Kp;
-      prow = P.tp + (size_t)grow * P.Kp;
       cur = lower_bound_row(trow, P.Kp, n * BN);
       nidx = trow[cur];
       np = prow[cur];
     }
+    const float zl2 = P.zl2;
 #pragma unroll 1
     for (int j = 0; j < BN / 64; ++j) {
       float v[64];
       __syncwarp();
       tmem_ld_32x32b_x64(taddr + j * 64, v);
       const int c0 = n * BN + j * 64;
+      const float2 zl2v = make_float2(zl2, zl2), nb = make_float2(-bias, -bias);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) v[i] = ex2_approx(fmaf(v[i], kLog2e, -bias));
+      for (int i = 0; i < 64; i += 2) {
+        const float2 e = __ffma2_rn(make_float2(v[i], v[i + 1]), zl2v, nb);
+        v[i] = ex2_approx(e.x);
+        v[i + 1] = ex2_approx(e.y);
+      }
       if (nidx < c0 + 64) {                 // a teacher column in this group (rare)
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
@@ -615,7 +636,11 @@ struct EpiDz {
       }
       uint32_t w[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]) ^ sgn;
+      for (int i = 0; i < 32; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+      if (sgn) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] ^= sgn;
+      }
       stage_store(cx, out, c0, cx.row_base, w, false);
     }
   }

@@ -5,10 +5,12 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 
 namespace kd {
 
 constexpr int kSentinel = 0x7fffffff;       // sorted-index padding; never equals a column
+constexpr int kEmptySlot = -1;              // teacher index of an empty cache slot
 constexpr int kMaxK = 512;
 constexpr int kPrepWarps = 4;               // tokens per block in teacher_prep
 constexpr int kMergeThreads = 256;
@@ -39,17 +41,21 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 }
 
 // One warp per token.  For token n it
-//  * turns the K cached logits into p = softmax(logit / T) and the teacher
-//    term sum_k p log p (0 log 0 = 0) -- the renormalised top-K teacher
-//    distribution of the offline cache;
-//  * drops (and counts) indices outside [0, V);
+//  * turns the cached logits of the filled slots into p = softmax(logit / T)
+//    and the teacher term sum_k p log p (0 log 0 = 0) -- the renormalised
+//    top-K teacher distribution of the offline cache.  A slot with index -1
+//    is empty and takes no part; a token without a finite filled logit gets
+//    p = 0 throughout (an empty teacher distribution);
+//  * drops (and counts) other indices outside [0, V);
 //  * sorts the (index, p) pairs by index (rank sort, ties by slot), merges
 //    repeated indices by adding their p, and writes the unique pairs padded
 //    with kSentinel to a row of Kp >= K + 1 slots, so the GEMM epilogues can
-//    walk a row's teacher columns in increasing order with one cursor.
-// Each block also writes the sum of its tokens' mask values (fp64).
+//    walk a row's teacher columns in increasing order with one cursor (and
+//    an empty distribution is a row that starts with kSentinel).
+// Logits are fp32, or bf16 when logit_bf16 != 0.  Each block also writes the
+// sum of its tokens' mask values (fp64).
 __global__ void __launch_bounds__(kPrepWarps * 32)
-teacher_prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ logit,
+teacher_prep_kernel(const int32_t* __restrict__ idx, const void* __restrict__ logit, int logit_bf16,
                     const float* __restrict__ mask, int N, int K, int Kp, int V, float T,
                     int32_t* __restrict__ tidx, float* __restrict__ tp, float* __restrict__ ent,
                     double* __restrict__ mask_part, Status* status) {
@@ -69,18 +75,23 @@ teacher_prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ l
   double mval = 0.0;
   if (n < N) {
     const int32_t* irow = idx + (size_t)n * K;
-    const float* lrow = logit + (size_t)n * K;
     float tmax = -INFINITY;
     for (int k = lane; k < K; k += 32) {
-      const float t = lrow[k] / T;
+      const float lg = logit_bf16
+          ? __bfloat162float(static_cast<const __nv_bfloat16*>(logit)[(size_t)n * K + k])
+          : static_cast<const float*>(logit)[(size_t)n * K + k];
+      const float t = irow[k] == kEmptySlot ? -INFINITY : lg / T;
       pv[k] = t;
       tmax = fmaxf(tmax, t);
     }
     tmax = warp_max(tmax);
-    float s = 0.f;
-    for (int k = lane; k < K; k += 32) s += expf(pv[k] - tmax);
-    s = warp_sum(s);
-    const float lse_t = tmax + logf(s);
+    float lse_t = INFINITY;                 // empty distribution: every p = 0
+    if (tmax != -INFINITY) {
+      float s = 0.f;
+      for (int k = lane; k < K; k += 32) s += expf(pv[k] - tmax);
+      s = warp_sum(s);
+      lse_t = tmax + logf(s);
+    }
     float e = 0.f;
     unsigned int nbad = 0;
     for (int k = lane; k < K; k += 32) {
@@ -89,7 +100,11 @@ teacher_prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ l
       if (p > 0.f) e += p * logp;
       int key_k = irow[k];
       float p_k = p;
-      if (key_k < 0 || key_k >= V) { key_k = kSentinel; p_k = 0.f; ++nbad; }
+      if (key_k < 0 || key_k >= V) {
+        nbad += key_k != kEmptySlot;
+        key_k = kSentinel;
+        p_k = 0.f;
+      }
       key[k] = key_k;
       pv[k] = p_k;
     }
@@ -147,14 +162,19 @@ teacher_prep_kernel(const int32_t* __restrict__ idx, const float* __restrict__ l
   }
 }
 
-// One thread per token: merge the per-split running (max, sum-exp, gathered
-// sum p*z) into lse and the token's KL term
-//   term = sum_k p log p - sum_k p z[idx_k] + lse      (sum_k p = 1),
-// and write each block's sum of mask * term (fp64).
+// One thread per token: merges the per-split (max, sum-exp, gathered p.z)
+// partials into lse and the token's KL term, and writes each block's sum of
+// mask * term (fp64).  The partials hold the maximum of the raw logits z and
+// sums of exp((z - max) * zscale), so the merged lse is that of z * zscale
+// (zscale = 1, or 1 / T for the student-temperature variant), and
+//   term = tfac * (sum p log p - zscale * sum p z + P * lse)
+// with P = 1, or 0 for a token without teacher entries (its prepared row
+// starts with kSentinel), and tfac = 1 or T^2.
 __global__ void __launch_bounds__(kMergeThreads)
 lse_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
                  const float* __restrict__ part_g, int splits, int N,
                  const float* __restrict__ ent, const float* __restrict__ mask,
+                 const int32_t* __restrict__ tidx, int Kp, float zscale, float tfac,
                  float* __restrict__ lse_out, double* __restrict__ term_part) {
   __shared__ double s_red[kMergeThreads / 32];
   const int n = blockIdx.x * kMergeThreads + threadIdx.x;
@@ -165,12 +185,13 @@ lse_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ par
     float ssum = 0.f, g = 0.f;
     for (int s = 0; s < splits; ++s) {
       const float ms = part_m[(size_t)s * N + n];
-      if (ms != -INFINITY) ssum += part_s[(size_t)s * N + n] * expf(ms - m);
+      if (ms != -INFINITY) ssum += part_s[(size_t)s * N + n] * expf((ms - m) * zscale);
       g += part_g[(size_t)s * N + n];
     }
-    const float lse = m + logf(ssum);
+    const float lse = m * zscale + logf(ssum);
     lse_out[n] = lse;
-    const float term = ent[n] - g + lse;
+    const float P = tidx[(size_t)n * Kp] == kSentinel ? 0.f : 1.f;
+    const float term = tfac * (ent[n] - zscale * g + P * lse);
     const float mv = mask ? mask[n] : 1.f;
     contrib = (mv != 0.f) ? (double)mv * (double)term : 0.0;
   }

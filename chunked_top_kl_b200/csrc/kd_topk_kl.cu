@@ -233,15 +233,41 @@ using ProbDz = Prob<EpiDz, false, false, kL2EvictLast, kL2Normal>;    // A = H c
 using ProbDh = Prob<EpiDh, false, true>;      // A = dZ (K-major over V), B = W (MN-major over d)
 using ProbDw = Prob<EpiDw, true, true, kL2Normal, kL2EvictLast>;      // A = dZ^T (MN-major over V), B = H chunk
 
-int common_checks(const void* H, const void* W, const int32_t* idx, const float* logit,
-                  int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+// The loss as one call computes it: the teacher logits and their type, T,
+// and the factors of the student-temperature variant (zs on the student
+// logits, T^2 on the term, T on dZ).
+struct Variant {
+  const void* logit;
+  int logit_bf16;
+  float T;
+  float zscale, tfac, gfac;
+};
+
+int make_variant(const kd_topk_kl_options* o, const void* logit, float T, Variant* v) {
+  kd_topk_kl_options d{};
+  if (o) d = *o;
+  if ((d.logit_bf16 | d.student_temperature) & ~1) return KD_ERR_INVALID_ARG;
+  for (int32_t r : d.reserved)
+    if (r) return KD_ERR_INVALID_ARG;
+  v->logit = logit;
+  v->logit_bf16 = d.logit_bf16;
+  v->T = T;
+  v->zscale = d.student_temperature ? 1.0f / T : 1.0f;
+  v->tfac = d.student_temperature ? T * T : 1.0f;
+  v->gfac = d.student_temperature ? T : 1.0f;
+  return KD_OK;
+}
+
+int common_checks(const void* H, const void* W, const int32_t* idx, const Variant& var,
+                  int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk,
                   void* ws, size_t ws_bytes, Layout* L) {
-  int st = check_shapes(N, d, V, K, T, chunk);
+  int st = check_shapes(N, d, V, K, var.T, chunk);
   if (st != KD_OK) return st;
   if (!W || !ws) return KD_ERR_INVALID_ARG;
-  if (N > 0 && (!H || !idx || !logit)) return KD_ERR_INVALID_ARG;
+  if (N > 0 && (!H || !idx || !var.logit)) return KD_ERR_INVALID_ARG;
   if (!aligned(W, 16) || (H && !aligned(H, 16)) || !aligned(ws, 256)) return KD_ERR_INVALID_ARG;
-  if ((idx && !aligned(idx, 4)) || (logit && !aligned(logit, 4))) return KD_ERR_INVALID_ARG;
+  if ((idx && !aligned(idx, 4)) || (var.logit && !aligned(var.logit, var.logit_bf16 ? 2 : 4)))
+    return KD_ERR_INVALID_ARG;
   *L = make_layout(N, V, K, chunk);
   if (ws_bytes < L->total) return KD_ERR_WORKSPACE;
   return KD_OK;
@@ -264,8 +290,8 @@ struct LaunchEvents {
 };
 
 
-int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
-                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const Variant& var,
+                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K,
                   const Layout& L, float* loss, float* lse, void* workspace, cudaStream_t s,
                   LaunchEvents& evs);
 
@@ -295,15 +321,26 @@ int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
                        const float* topk_logit, const float* mask, int64_t N, int64_t d,
                        int64_t V, int64_t K, float T, int64_t chunk, float* loss, float* lse,
                        void* workspace, size_t workspace_bytes, void* stream) {
+  return kd_topk_kl_forward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, loss, lse,
+                               workspace, workspace_bytes, stream, nullptr);
+}
+
+int kd_topk_kl_forward_ex(const void* H, const void* W, const int32_t* topk_idx,
+                          const void* topk_logit, const float* mask, int64_t N, int64_t d,
+                          int64_t V, int64_t K, float T, int64_t chunk, float* loss, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          const kd_topk_kl_options* options) {
+  Variant var;
+  int st = make_variant(options, topk_logit, T, &var);
+  if (st != KD_OK) return st;
   Layout L;
-  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
-                         workspace_bytes, &L);
+  st = common_checks(H, W, topk_idx, var, N, d, V, K, chunk, workspace, workspace_bytes, &L);
   if (st != KD_OK) return st;
   if (!loss || (N > 0 && !lse)) return KD_ERR_INVALID_ARG;
   if (mask && !aligned(mask, 4)) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchEvents evs{nullptr, 0, 0, s};
-  return forward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, L, loss, lse, workspace, s, evs);
+  return forward_stage(H, W, topk_idx, var, mask, N, d, V, K, L, loss, lse, workspace, s, evs);
 }
 
 }  // extern "C"
@@ -312,8 +349,8 @@ namespace {
 
 // Forward pass on a checked workspace layout: clears the status words, then
 // teacher prep, the logits/lse GEMM, the lse merge and the loss.
-int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
-                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const Variant& var,
+                  const float* mask, int64_t N, int64_t d, int64_t V, int64_t K,
                   const Layout& L, float* loss, float* lse, void* workspace, cudaStream_t s,
                   LaunchEvents& evs) {
   int dev = 0;
@@ -333,7 +370,8 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const f
 
   if (!evs.mark()) return KD_ERR_CUDA;
   teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
-      topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+      topk_idx, var.logit, var.logit_bf16, mask, (int)N, (int)K, L.Kp, (int)V, var.T, tidx, tp, ent,
+      mask_part, status);
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
 
   CUtensorMap tmH, tmW;
@@ -348,6 +386,7 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const f
   ep.N = (int)N;
   ep.V = (int)V;
   ep.Kp = L.Kp;
+  ep.zl2 = var.zscale * kLog2e;
   ep.tidx = tidx;
   ep.tp = tp;
   ep.part_m = at<float>(workspace, L.off_pm);
@@ -359,7 +398,8 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const f
 
   if (!evs.mark()) return KD_ERR_CUDA;
   lse_merge_kernel<<<(unsigned)L.n_merge_blocks, kMergeThreads, 0, s>>>(
-      ep.part_m, ep.part_s, ep.part_g, a.raster.splits, (int)N, ent, mask, lse, term_part);
+      ep.part_m, ep.part_s, ep.part_g, a.raster.splits, (int)N, ent, mask, tidx, L.Kp, var.zscale,
+      var.tfac, lse, term_part);
   if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, term_part,
                                     (int)L.n_merge_blocks, 0, nullptr, loss);
@@ -379,8 +419,8 @@ int backward_checks(int64_t N, const float* lse, const float* grad_loss, const f
 // words are cleared and the teacher cache is prepared here; without it the
 // forward pass of the same call has done both.  Then the gradient scale and,
 // per chunk, the dZ recompute and the joint dH / dW launch.
-int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const float* topk_logit,
-                   const float* mask, int64_t N, int64_t d, int64_t V, int64_t K, float T,
+int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const Variant& var,
+                   const float* mask, int64_t N, int64_t d, int64_t V, int64_t K,
                    int64_t chunk, const Layout& L, const float* lse, const float* grad_loss,
                    void* dH, float* dW, int accumulate_dW, void* workspace, cudaStream_t s,
                    bool run_prep, LaunchEvents& evs) {
@@ -404,7 +444,8 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
   if (run_prep) {
     if (!evs.mark()) return KD_ERR_CUDA;
     teacher_prep_kernel<<<(unsigned)L.n_prep_blocks, kPrepWarps * 32, 0, s>>>(
-        topk_idx, topk_logit, mask, (int)N, (int)K, L.Kp, (int)V, T, tidx, tp, ent, mask_part, status);
+        topk_idx, var.logit, var.logit_bf16, mask, (int)N, (int)K, L.Kp, (int)V, var.T, tidx, tp, ent,
+        mask_part, status);
   }
   if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, nullptr, 0, 1, grad_loss, cscale);
@@ -436,6 +477,8 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     e3.V = (int)V;
     e3.ldz = (int)L.ldz;
     e3.Kp = L.Kp;
+    e3.zl2 = var.zscale * kLog2e;
+    e3.gfac = var.gfac;
     e3.tidx = tidx;
     e3.tp = tp;
     e3.lse = lse;
@@ -477,9 +520,9 @@ int kd_topk_kl_backward(const void* H, const void* W, const int32_t* topk_idx,
                         int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
                         const float* grad_loss, void* dH, float* dW, int accumulate_dW,
                         void* workspace, size_t workspace_bytes, void* stream) {
-  return kd_topk_kl_backward_profiled(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse,
-                                      grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes,
-                                      stream, nullptr, 0);
+  return kd_topk_kl_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse,
+                                grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes,
+                                stream, nullptr, 0, nullptr);
 }
 
 int kd_topk_kl_backward_profiled(const void* H, const void* W, const int32_t* topk_idx,
@@ -488,17 +531,31 @@ int kd_topk_kl_backward_profiled(const void* H, const void* W, const int32_t* to
                                  const float* grad_loss, void* dH, float* dW, int accumulate_dW,
                                  void* workspace, size_t workspace_bytes, void* stream,
                                  void* const* events, int64_t n_events) {
+  return kd_topk_kl_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, lse,
+                                grad_loss, dH, dW, accumulate_dW, workspace, workspace_bytes,
+                                stream, events, n_events, nullptr);
+}
+
+int kd_topk_kl_backward_ex(const void* H, const void* W, const int32_t* topk_idx,
+                           const void* topk_logit, const float* mask, int64_t N, int64_t d,
+                           int64_t V, int64_t K, float T, int64_t chunk, const float* lse,
+                           const float* grad_loss, void* dH, float* dW, int accumulate_dW,
+                           void* workspace, size_t workspace_bytes, void* stream,
+                           void* const* events, int64_t n_events,
+                           const kd_topk_kl_options* options) {
+  Variant var;
+  int st = make_variant(options, topk_logit, T, &var);
+  if (st != KD_OK) return st;
   Layout L;
-  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
-                         workspace_bytes, &L);
+  st = common_checks(H, W, topk_idx, var, N, d, V, K, chunk, workspace, workspace_bytes, &L);
   if (st != KD_OK) return st;
   if ((st = backward_checks(N, lse, grad_loss, mask, dH, dW)) != KD_OK) return st;
   const int64_t launches = N > 0 ? 2 + 2 * ceil_div(N, chunk) : 0;
   if (events && n_events < launches + 1) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
-  st = backward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, L, lse, grad_loss, dH,
-                      dW, accumulate_dW, workspace, s, true, evs);
+  st = backward_stage(H, W, topk_idx, var, mask, N, d, V, K, chunk, L, lse, grad_loss, dH, dW,
+                      accumulate_dW, workspace, s, true, evs);
   if (st == KD_OK && N > 0 && !evs.mark()) return KD_ERR_CUDA;
   return st;
 }
@@ -509,9 +566,23 @@ int kd_topk_kl_forward_backward(const void* H, const void* W, const int32_t* top
                                 float* lse, const float* grad_loss, void* dH, float* dW,
                                 int accumulate_dW, void* workspace, size_t workspace_bytes,
                                 void* stream, void* const* events, int64_t n_events) {
+  return kd_topk_kl_forward_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, loss,
+                                        lse, grad_loss, dH, dW, accumulate_dW, workspace,
+                                        workspace_bytes, stream, events, n_events, nullptr);
+}
+
+int kd_topk_kl_forward_backward_ex(const void* H, const void* W, const int32_t* topk_idx,
+                                   const void* topk_logit, const float* mask, int64_t N,
+                                   int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                                   float* loss, float* lse, const float* grad_loss, void* dH,
+                                   float* dW, int accumulate_dW, void* workspace,
+                                   size_t workspace_bytes, void* stream, void* const* events,
+                                   int64_t n_events, const kd_topk_kl_options* options) {
+  Variant var;
+  int st = make_variant(options, topk_logit, T, &var);
+  if (st != KD_OK) return st;
   Layout L;
-  int st = common_checks(H, W, topk_idx, topk_logit, N, d, V, K, T, chunk, workspace,
-                         workspace_bytes, &L);
+  st = common_checks(H, W, topk_idx, var, N, d, V, K, chunk, workspace, workspace_bytes, &L);
   if (st != KD_OK) return st;
   if (!loss || (N > 0 && !lse)) return KD_ERR_INVALID_ARG;
   if ((st = backward_checks(N, lse, grad_loss, mask, dH, dW)) != KD_OK) return st;
@@ -519,10 +590,10 @@ int kd_topk_kl_forward_backward(const void* H, const void* W, const int32_t* top
   if (events && n_events < launches + 1) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
-  st = forward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, L, loss, lse, workspace, s, evs);
+  st = forward_stage(H, W, topk_idx, var, mask, N, d, V, K, L, loss, lse, workspace, s, evs);
   if (st != KD_OK) return st;
-  st = backward_stage(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, chunk, L, lse, grad_loss, dH,
-                      dW, accumulate_dW, workspace, s, false, evs);
+  st = backward_stage(H, W, topk_idx, var, mask, N, d, V, K, chunk, L, lse, grad_loss, dH, dW,
+                      accumulate_dW, workspace, s, false, evs);
   if (st == KD_OK && N > 0 && !evs.mark()) return KD_ERR_CUDA;
   return st;
 }

@@ -24,6 +24,22 @@
  * T divides the teacher logits only.  Duplicate teacher indices add their
  * probabilities at that column (the loss keeps the per-slot sum).
  *
+ * A teacher index of -1 marks an empty cache slot (a cache that holds fewer
+ * than K entries for some tokens): the slot takes no part in the teacher
+ * softmax, so p is renormalised over the filled slots.  A token without a
+ * filled slot (or whose filled logits are all -inf) has an empty teacher
+ * distribution: term = 0 and a zero dZ row (d term / dz = P softmax(z) -
+ * scatter(p) with P = sum_k p = 0); its mask still counts in sum m.
+ *
+ * Variants selected through kd_topk_kl_options (the *_ex entry points; the
+ * pages describe neither):
+ *  - logit_bf16: topk_logit holds bf16 values instead of fp32.
+ *  - student_temperature: the usual distillation temperature on both sides:
+ *      lse[n]  = log sum_v exp(z[n,v] / T)
+ *      term[n] = T^2 sum_k p (log p - (z[n,idx]/T - lse[n]))
+ *      dZ[n,v] = g m[n] / sum m * T (exp(z[n,v]/T - lse[n]) - scatter(p))
+ *    lse is then that of z / T, and the backward pass must be given it.
+ *
  * Conventions shared by every entry point:
  *  - All array pointers are DEVICE pointers owned by the caller.  No call
  *    allocates device or host memory.  The library keeps no state between
@@ -40,10 +56,10 @@
  *  - Supported shapes: N >= 0, 1 <= V < 2^31, d >= 8 with d % 8 == 0,
  *    1 <= K <= 512, T > 0 and finite, chunk >= 1.  H, W, dH and dW must be
  *    16-byte aligned, the workspace 256-byte aligned.
- *  - Teacher indices outside [0, V) are not an argument error: they are
- *    dropped (contribute nothing), counted in the workspace and reported by
- *    kd_topk_kl_check as KD_ERR_BAD_INDEX; the results are then undefined
- *    in value but every memory access stays in bounds.
+ *  - Teacher indices outside [0, V) other than -1 are not an argument
+ *    error: they are dropped (contribute nothing), counted in the workspace
+ *    and reported by kd_topk_kl_check as KD_ERR_BAD_INDEX; the results are
+ *    then undefined in value but every memory access stays in bounds.
  *  - Results are deterministic: the same inputs give bitwise the same
  *    outputs on every run (fixed-order reductions, no float atomics).
  *  - A workspace may be used by one call at a time (calls on one stream
@@ -172,6 +188,50 @@ int kd_topk_kl_forward_noalloc(const void* H, const void* W,
                                const float* mask,
                                int64_t N, int64_t d, int64_t V, int64_t K, float T,
                                float* loss, float* lse, void* stream);
+
+/* Options of the *_ex entry points.  A NULL pointer, or a zero-filled
+ * struct, selects the definition above (fp32 logits, T on the teacher
+ * only).  Every field is 0 or 1; reserved fields must be 0, else
+ * KD_ERR_INVALID_ARG. */
+typedef struct kd_topk_kl_options {
+  int32_t logit_bf16;           /* 1: topk_logit is bf16 [N][K] (2-byte aligned) */
+  int32_t student_temperature;  /* 1: student logits divided by T too, term times T^2 */
+  int32_t reserved[6];
+} kd_topk_kl_options;
+
+/* kd_topk_kl_forward with options; topk_logit is fp32 or bf16 as
+ * options->logit_bf16 says. */
+int kd_topk_kl_forward_ex(const void* H, const void* W,
+                          const int32_t* topk_idx, const void* topk_logit,
+                          const float* mask,
+                          int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                          float* loss, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          const kd_topk_kl_options* options);
+
+/* kd_topk_kl_backward_profiled with options (events may be NULL).  With
+ * student_temperature, lse must come from a forward pass with the same
+ * options. */
+int kd_topk_kl_backward_ex(const void* H, const void* W,
+                           const int32_t* topk_idx, const void* topk_logit,
+                           const float* mask,
+                           int64_t N, int64_t d, int64_t V, int64_t K, float T, int64_t chunk,
+                           const float* lse, const float* grad_loss,
+                           void* dH, float* dW, int accumulate_dW,
+                           void* workspace, size_t workspace_bytes, void* stream,
+                           void* const* events, int64_t n_events,
+                           const kd_topk_kl_options* options);
+
+/* kd_topk_kl_forward_backward with options. */
+int kd_topk_kl_forward_backward_ex(const void* H, const void* W,
+                                   const int32_t* topk_idx, const void* topk_logit,
+                                   const float* mask,
+                                   int64_t N, int64_t d, int64_t V, int64_t K, float T,
+                                   int64_t chunk, float* loss, float* lse, const float* grad_loss,
+                                   void* dH, float* dW, int accumulate_dW,
+                                   void* workspace, size_t workspace_bytes, void* stream,
+                                   void* const* events, int64_t n_events,
+                                   const kd_topk_kl_options* options);
 
 /* Synchronises `stream`, then reads the device-side status words that the
  * last forward or backward call on this workspace wrote.  Returns KD_OK,

@@ -90,3 +90,26 @@ def test_argument_errors_are_synchronous(lib):
     assert B(P, P, P, P, None, N, d, V, K, 1.0, 128, P, None, P, None, 0, P, nb, None) == _abi.KD_ERR_INVALID_ARG
     assert B(P, P, P, P, None, N, d, V, K, 1.0, 128, P, None, P + 4, P, 0, P, nb, None) == _abi.KD_ERR_INVALID_ARG
     assert B(P, P, P, P, None, N, d, V, K, 1.0, 128, None, None, P, P, 0, P, nb, None) == _abi.KD_ERR_INVALID_ARG
+
+
+def test_options_are_validated_first(lib):
+    from chunked_top_kl_b200 import _abi
+    P = 1 << 20          # never dereferenced: the options are rejected before any other check
+    N, d, V, K = 512, 256, 4096, 16
+    nb = lib.kd_topk_kl_workspace_size(N, d, V, K, 128)
+
+    def fwd(opt, logit=P):
+        return _abi.kd_topk_kl_forward_ex(P, P, P, logit, None, N, d, V, K, 1.0, 128, P, P, P, nb, None, opt)
+
+    bad = _abi.make_options()
+    bad.reserved[3] = 1
+    assert fwd(bad) == _abi.KD_ERR_INVALID_ARG
+    bad = _abi.make_options()
+    bad.student_temperature = 2
+    assert fwd(bad) == _abi.KD_ERR_INVALID_ARG
+    assert _abi.kd_topk_kl_backward_ex(P, P, P, P, None, N, d, V, K, 1.0, 128, P, None, P, P, 0, P, nb,
+                                       None, None, bad) == _abi.KD_ERR_INVALID_ARG
+    assert _abi.kd_topk_kl_forward_backward_ex(P, P, P, P, None, N, d, V, K, 1.0, 128, P, P, None, P, P, 0,
+                                               P, nb, None, None, bad) == _abi.KD_ERR_INVALID_ARG
+    # fp32 logits need 4-byte alignment (rejected before anything is enqueued)
+    assert fwd(_abi.make_options(), logit=P + 2) == _abi.KD_ERR_INVALID_ARG
