@@ -161,32 +161,49 @@ def barrier(world: int):
         dist.barrier()
 
 
-def launches_per_step(N: int, chunk: int) -> int:
+# Below this many tokens the row compaction and the per-chunk gather/scatter
+# launches cost about what skipping the masked rows saves.
+AUTO_SKIP_MIN_N = 16384
+
+
+def launches_per_step(N: int, chunk: int, skip_rows: bool = False) -> int:
     """Kernels this library launches for one fused forward+backward call:
     teacher prep, logits/lse GEMM, lse merge, loss, gradient scale, and per
-    chunk the dZ recompute GEMM and the joint dH/dW GEMM."""
+    chunk the dZ recompute GEMM and the joint dH/dW GEMM; when masked rows are
+    skipped, also the row compaction and per chunk a row gather and scatter."""
     if N == 0:
         return 0
-    return 5 + 2 * math.ceil(N / chunk)
+    c = math.ceil(N / chunk)
+    return 6 + 4 * c if skip_rows else 5 + 2 * c
 
 
-def per_kernel_times(ev, N, d, V, chunk):
+def per_kernel_times(ev, N, d, V, chunk, kept=None):
     """Live per-kernel totals from the events recorded around every launch of
     the fused call: 0 teacher prep, 1 logits/lse GEMM, 2 lse merge, 3 loss,
     4 gradient scale, then per chunk c the dZ recompute (5+2c) and the joint
-    dH/dW GEMM (6+2c)."""
+    dH/dW GEMM (6+2c).  With skipped rows (`kept` = tokens the backward
+    processes): 5 row compaction, then per chunk the row gather (6+4c), dZ
+    recompute (7+4c), joint dH/dW GEMM (8+4c) and dH row scatter (9+4c); the
+    GEMMs' flops count the kept rows of each chunk only."""
     names = {0: ("teacher_prep", 0.0), 1: ("forward_gemm", 2.0 * N * d * V), 2: ("lse_merge", 0.0),
              3: ("loss", 0.0), 4: ("grad_scale", 0.0)}
+    if kept is not None:
+        names[5] = ("row_compaction", 0.0)
     out = {}
     for row in ev:
         for j in range(len(row) - 1):
             if j in names:
                 key, flops = names[j]
-            else:
+            elif kept is None:
                 c = (j - 5) // 2
                 cc = min(chunk, N - c * chunk)
                 key, flops = (("dz_recompute", 2.0 * cc * d * V) if (j - 5) % 2 == 0
                               else ("grads_dH_dW", 4.0 * cc * d * V))
+            else:
+                c, r = divmod(j - 6, 4)
+                cc = max(0, min(chunk, kept - c * chunk))
+                key, flops = [("row_gather", 0.0), ("dz_recompute", 2.0 * cc * d * V),
+                              ("grads_dH_dW", 4.0 * cc * d * V), ("row_scatter", 0.0)][r]
             k = out.setdefault(key, {"launches": 0, "ms": 0.0, "flops": 0.0})
             k["launches"] += 1
             k["ms"] += row[j].elapsed_time(row[j + 1])
@@ -277,9 +294,13 @@ def run_cuda(args, cfg, world, rank, local):
     dW = torch.empty((V, d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    n_kept = int(((x["mask"] != 0) & (x["topk_idx"] != -1).any(dim=1)).sum())
+    skip = args.backward_rows == "kept" or (args.backward_rows == "auto" and n_kept < N and N >= AUTO_SKIP_MIN_N)
+    kept = n_kept if skip else None
+
     def step():
         loss, _, _, _ = kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T,
-                                            chunk, workspace=ws, dH=dH, dW=dW)
+                                            chunk, workspace=ws, dH=dH, dW=dW, skip_masked_rows=skip)
         return loss
 
     for _ in range(args.warmup):
@@ -295,7 +316,7 @@ def run_cuda(args, cfg, world, rank, local):
     # fused forward+backward call that records an event before each of its
     # kernel launches and after the last (same kernels and work as without
     # events), which gives live per-kernel durations on the launching stream.
-    nl = kd.forward_backward_launches(N, chunk)
+    nl = kd.forward_backward_launches(N, chunk, skip)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(args.steps)]
     for row in ev:
         for e in row:
@@ -311,13 +332,13 @@ def run_cuda(args, cfg, world, rank, local):
     start.record(stream)
     for i in range(args.steps):
         kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk,
-                            workspace=ws, dH=dH, dW=dW, events=ev[i])
+                            workspace=ws, dH=dH, dW=dW, events=ev[i], skip_masked_rows=skip)
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     clocks = sampler.stop() if sampler else None
     ms_local = start.elapsed_time(end)
-    kern = per_kernel_times(ev, N, d, V, chunk)
+    kern = per_kernel_times(ev, N, d, V, chunk, kept)
     ms = reduce_max(ms_local, world, dev)
     st, _ = kd.check(ws)
     if st != 0:
@@ -363,7 +384,8 @@ def run_cuda(args, cfg, world, rank, local):
     dom_name, dom = max(((k, v) for k, v in kern.items() if v["flops"] > 0), key=lambda kv: kv[1]["ms"])
     dom_ach = dom["tflops"]
     fwd_avg = sum(kern[k]["ms"] for k in ("teacher_prep", "forward_gemm", "lse_merge", "loss")) / args.steps
-    bwd_avg = sum(kern[k]["ms"] for k in ("grad_scale", "dz_recompute", "grads_dH_dW")) / args.steps
+    bwd_avg = sum(v["ms"] for k, v in kern.items()
+                  if k not in ("teacher_prep", "forward_gemm", "lse_merge", "loss")) / args.steps
     peak_sus = peaks["bf16_tflops_sustained"]
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -381,9 +403,9 @@ def run_cuda(args, cfg, world, rank, local):
         "pct_bf16_peak_sustained": tflops / world / peak_sus,
         "peak_hbm_gib": peak_gib, "workspace_gib": ws_gib,
         "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
-        "config": config_block(cfg, world),
+        "config": {**config_block(cfg, world), "backward_rows": "kept tokens only" if skip else "all tokens"},
         "clocks": clocks,
-        "gpu_launches": launches_per_step(N, chunk) * args.steps,
+        "gpu_launches": launches_per_step(N, chunk, skip) * args.steps,
         "roofline": {"bound": "tensor", "kernel": dom_name,
                      "achieved": dom_ach, "peak": peak_sus, "unit": "TFLOP/s", "frac": dom_ach / peak_sus,
                      "peak_kind": f"bf16_tflops_sustained ({peaks_src})",
@@ -413,6 +435,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--backward-rows", choices=["auto", "all", "kept"], default="auto",
+                    help="backward over every token, or over the tokens with a non-zero dZ row only "
+                         "(same results; auto: kept when some token is masked and N >= %d)" % AUTO_SKIP_MIN_N)
     ap.add_argument("--cpu-flops", type=float, default=4e12, help="oracle work for cpu_baseline")
     ap.add_argument("--ref-flops", type=float, default=1.2e12, help="oracle work per reference step")
     args = ap.parse_args(argv)

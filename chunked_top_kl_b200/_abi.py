@@ -38,13 +38,15 @@ EXPORTS = (
 class KDOptions(ctypes.Structure):
     """kd_topk_kl_options (see the C header)."""
     _fields_ = [("logit_bf16", ctypes.c_int32), ("student_temperature", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("skip_masked_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
 
 
-def make_options(logit_bf16: bool = False, student_temperature: bool = False) -> KDOptions:
+def make_options(logit_bf16: bool = False, student_temperature: bool = False,
+                 skip_masked_rows: bool = False) -> KDOptions:
     o = KDOptions()
     o.logit_bf16 = int(bool(logit_bf16))
     o.student_temperature = int(bool(student_temperature))
+    o.skip_masked_rows = int(bool(skip_masked_rows))
     return o
 
 

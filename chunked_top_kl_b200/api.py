@@ -53,13 +53,26 @@ def _raise(st: int, where: str):
         raise _abi.KDError(st, where)
 
 
-def _options(topk_logit, student_temperature: bool):
-    """kd_topk_kl_options for these inputs, or None for the default loss
-    (fp32 logits, T on the teacher only): the plain entry points then run."""
-    bf16 = topk_logit.dtype == torch.bfloat16
-    if not bf16 and not student_temperature:
+def _event_handles(events):
+    """cudaEvent_t handles of torch.cuda.Event objects; an Event creates its
+    CUDA event on first record, so a fresh one is recorded once here."""
+    if events is None:
         return None
-    return _abi.make_options(logit_bf16=bf16, student_temperature=student_temperature)
+    for e in events:
+        if not e.cuda_event:
+            e.record()
+    return [e.cuda_event for e in events]
+
+
+def _options(topk_logit, student_temperature: bool, skip_masked_rows: bool = False):
+    """kd_topk_kl_options for these inputs, or None for the default loss
+    (fp32 logits, T on the teacher only, every row): the plain entry points
+    then run."""
+    bf16 = topk_logit.dtype == torch.bfloat16
+    if not bf16 and not student_temperature and not skip_masked_rows:
+        return None
+    return _abi.make_options(logit_bf16=bf16, student_temperature=student_temperature,
+                             skip_masked_rows=skip_masked_rows)
 
 
 def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
@@ -89,20 +102,23 @@ def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 
     return loss, lse
 
 
-def backward_launches(N: int, chunk: int) -> int:
+def backward_launches(N: int, chunk: int, skip_masked_rows: bool = False) -> int:
     """Kernel launches of one backward call (see kd_topk_kl_backward_profiled)."""
-    return 0 if N == 0 else 2 + 2 * ((N + chunk - 1) // chunk)
+    c = (N + chunk - 1) // chunk
+    return 0 if N == 0 else (3 + 4 * c if skip_masked_rows else 2 + 2 * c)
 
 
 def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.Tensor,
              grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
              accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
              dH: Optional[torch.Tensor] = None, events=None,
-             student_temperature: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+             student_temperature: bool = False,
+             skip_masked_rows: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Returns (dH [N,d] bf16, dW [V,d] fp32).  With ``events`` (a list of
     backward_launches(N, chunk) + 1 created torch.cuda.Event objects) the
     library records them around each of its kernel launches.
-    ``student_temperature`` must match the forward call that made ``lse``."""
+    ``student_temperature`` must match the forward call that made ``lse``;
+    ``skip_masked_rows`` skips the rows of tokens with a zero dZ row."""
     N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
     dev = H.device
     if workspace is None:
@@ -115,13 +131,13 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
     if grad_loss is not None:
         grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    opt = _options(topk_logit, student_temperature)
+    opt = _options(topk_logit, student_temperature, skip_masked_rows)
     if opt is not None:
         st = _abi.kd_topk_kl_backward_ex(
             _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
             int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
             _ptr(workspace), workspace.numel(), stream,
-            None if events is None else [e.cuda_event for e in events], opt)
+            _event_handles(events), opt)
         _raise(st, "kd_topk_kl_backward_ex")
     elif events is None:
         st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
@@ -133,20 +149,22 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
         st = _abi.kd_topk_kl_backward_profiled(
             _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
             int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
-            _ptr(workspace), workspace.numel(), stream, [e.cuda_event for e in events])
+            _ptr(workspace), workspace.numel(), stream, _event_handles(events))
         _raise(st, "kd_topk_kl_backward_profiled")
     return dH, dW
 
 
-def forward_backward_launches(N: int, chunk: int) -> int:
+def forward_backward_launches(N: int, chunk: int, skip_masked_rows: bool = False) -> int:
     """Kernel launches of one fused forward + backward call."""
-    return 0 if N == 0 else 5 + 2 * ((N + chunk - 1) // chunk)
+    c = (N + chunk - 1) // chunk
+    return 0 if N == 0 else (6 + 4 * c if skip_masked_rows else 5 + 2 * c)
 
 
 def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 4096,
                      grad_loss: Optional[torch.Tensor] = None, dW: Optional[torch.Tensor] = None,
                      accumulate_dW: bool = False, workspace: Optional[torch.Tensor] = None,
-                     dH: Optional[torch.Tensor] = None, events=None, student_temperature: bool = False):
+                     dH: Optional[torch.Tensor] = None, events=None, student_temperature: bool = False,
+                     skip_masked_rows: bool = False):
     """One call for a training step: returns (loss, lse, dH, dW)."""
     N, d, V, K = _check_inputs(H, W, topk_idx, topk_logit, mask)
     dev = H.device
@@ -162,8 +180,8 @@ def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chun
     if grad_loss is not None:
         grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
     stream = torch.cuda.current_stream(dev).cuda_stream
-    evs = None if events is None else [e.cuda_event for e in events]
-    opt = _options(topk_logit, student_temperature)
+    evs = _event_handles(events)
+    opt = _options(topk_logit, student_temperature, skip_masked_rows)
     args = (_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T), int(chunk),
             _ptr(loss), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
             _ptr(workspace), workspace.numel(), stream)

@@ -62,6 +62,19 @@ struct ProbArgs {
   int num_kb;           // BK-wide K blocks per tile
   int a_row0, b_row0;   // added to the row (M / N) coordinate
   int a_k0, b_k0;       // added to the K coordinate
+  int dyn_role;         // with GemmArgs::dyn: 1 = the live rows are this GEMM's M, 2 = its K
+  int dyn_bands_fastest;
+  int dyn_zero_fill;    // role 2 with no live rows: still write the (zero) output tiles
+};
+
+// A launch over rows whose number is known only on the device (a chunk of the
+// compacted token list): the host plans `chunk` rows; every thread of the
+// kernel reads the live total and rebuilds the schedule for
+// clamp(*count - row0, 0, chunk) rows.
+struct DynRows {
+  const int* count;     // null: a static launch
+  int row0;
+  int chunk;
 };
 
 // A launch runs problem 0 and, optionally, problem 1.  Problem 0's units go
@@ -71,8 +84,28 @@ struct ProbArgs {
 struct GemmArgs {
   ProbArgs prob[2];
   JointPlan joint;
+  DynRows dyn;
   Status* status;
 };
+
+// The schedule of a launch with live row count `rows` (see DynRows).
+template <class G, bool HAS_P1>
+__device__ __forceinline__ void apply_live_rows(GemmArgs& a, int rows, int ngroups) {
+#pragma unroll
+  for (int p = 0; p < (HAS_P1 ? 2 : 1); ++p) {
+    ProbArgs& pa = a.prob[p];
+    if (pa.dyn_role == 1) {
+      pa.raster = tile_raster(ceil_div64(rows, G::TILE_M), pa.raster.n_tiles, pa.dyn_bands_fastest != 0);
+    } else if (pa.dyn_role == 2) {
+      pa.num_kb = (int)ceil_div64(rows, BK);
+      if (rows == 0 && !pa.dyn_zero_fill) pa.raster.num_units = 0;
+    }
+  }
+  if constexpr (HAS_P1)
+    a.joint = joint_plan(a.prob[0].raster.num_units, (int64_t)a.prob[0].raster.tiles_per_split * a.prob[0].num_kb,
+                         a.prob[1].raster.num_units, (int64_t)a.prob[1].raster.tiles_per_split * a.prob[1].num_kb,
+                         ngroups);
+}
 
 // Compile-time description of a problem: its epilogue, operand majorness,
 // and the L2 eviction priority of each operand's loads (L2Hint).
@@ -132,6 +165,7 @@ struct EpiCtx {
   int row_base;
   bool issuer;
   uint32_t seq;
+  int rows_valid;       // live rows of a DynRows launch, else -1
 };
 
 // Writes one 128-byte segment per thread (its row) into the next staging
@@ -357,6 +391,7 @@ __device__ __forceinline__ EpiCtx make_epi_ctx(uint32_t staging) {
   cx.issuer = (threadIdx.x == 64);
   cx.seq = 0;
   cx.row_base = 0;
+  cx.rows_valid = -1;
   return cx;
 }
 
@@ -389,15 +424,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   }
   const uint32_t tmem_base = pipeline_setup<G, PAIR>(L);
 
-  // This group's units: problem 0 round-robin, then problem 1's range.
+  // The schedule; a launch over a device-side row count rebuilds it here.
+  GemmArgs A = args;
+  int live_rows = -1;
+  if (args.dyn.count) {
+    int r = *args.dyn.count - args.dyn.row0;
+    r = r < 0 ? 0 : (r > args.dyn.chunk ? args.dyn.chunk : r);
+    live_rows = r;
+    apply_live_rows<G, P1::present>(A, r, ngroups);
+  }
+
+  // This group's units: problem 0 round-robin, then its share of problem 1.
   auto for_each_unit = [&](auto&& body) {
     bool ok = true;
-    for (int u = group; ok && u < args.prob[0].raster.num_units; u += ngroups)
-      ok = body(P0{}, args.prob[0], &tmA0, &tmB0, u);
+    for (int u = group; ok && u < A.prob[0].raster.num_units; u += ngroups)
+      ok = body(P0{}, A.prob[0], &tmA0, &tmB0, u);
     if constexpr (P1::present) {
-      const int n1 = joint_count(args.joint, args.prob[1].raster.num_units, ngroups, group);
+      const int n1 = joint_count(A.joint, A.prob[1].raster.num_units, ngroups, group);
       for (int i = 0; ok && i < n1; ++i)
-        ok = body(P1{}, args.prob[1], &tmA1, &tmB1, joint_unit(args.joint, ngroups, group, i));
+        ok = body(P1{}, A.prob[1], &tmA1, &tmB1, joint_unit(A.joint, ngroups, group, i));
     }
     return ok;
   };
@@ -421,6 +466,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     typename P0::Epi epi0;
     typename P1::Epi epi1;
     EpiCtx cx = make_epi_ctx(L.staging);
+    cx.rows_valid = live_rows;
     failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap*, const CUtensorMap*,
                                 int u) {
       using P = decltype(pt);
@@ -430,7 +476,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     });
     if (cx.issuer) bulk_wait<0>();          // every TMA store of this CTA has completed
   }
-  pipeline_teardown<G, PAIR>(L, failed, args.status, tmem_base);
+  pipeline_teardown<G, PAIR>(L, failed, A.status, tmem_base);
 }
 
 // ---------------------------------------------------------------- epilogues
@@ -569,6 +615,7 @@ struct EpiDz {
     int V, ldz, Kp;
     float zl2;             // zs log2(e)
     float gfac;            // 1, or T
+    const int32_t* rowmap; // null, or chunk row r is token rowmap[row0 + r]
     const int32_t* tidx;
     const float* tp;
     const float* lse;
@@ -580,8 +627,8 @@ struct EpiDz {
 
   __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int r, int n,
                                        uint32_t taddr, EpiCtx& cx) {
-    const bool valid = r < P.rows_valid;
-    const int grow = P.row0 + r;
+    const bool valid = r < (cx.rows_valid >= 0 ? cx.rows_valid : P.rows_valid);
+    const int grow = valid && P.rowmap ? P.rowmap[P.row0 + r] : P.row0 + r;
     // c exp(z zs - lse) = 2^(z zl2 - bias) with bias = lse log2(e) - log2(c):
     // one FFMA and one ex2 per element.  c = 0 (masked token, token without
     // teacher entries) and rows past the chunk give bias = +inf, hence exact
@@ -685,11 +732,18 @@ struct EpiDw {
 
   __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int, int n,
                                        uint32_t taddr, EpiCtx& cx) {
+    // A launch with no live rows (DynRows) ran no MMA: the tile is zero.
+    const bool empty = cx.rows_valid == 0;
 #pragma unroll 1
     for (int j = 0; j < BN / 32; ++j) {
       float v[32];
       __syncwarp();
-      tmem_ld_32x32b_x32(taddr + j * 32, v);
+      if (empty) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      } else {
+        tmem_ld_32x32b_x32(taddr + j * 32, v);
+      }
       uint32_t w[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);

@@ -205,6 +205,69 @@ lse_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ par
   }
 }
 
+// Rows that can be skipped in the backward pass: a token whose mask is 0, or
+// whose teacher distribution is empty, has a zero dZ row.  One block lists
+// the other tokens in increasing order in rowmap[0, *count) (a block-wide
+// exclusive scan of per-thread counts over contiguous token segments).
+constexpr int kCompactThreads = 1024;
+
+__global__ void __launch_bounds__(kCompactThreads)
+compact_rows_kernel(const float* __restrict__ mask, const int32_t* __restrict__ tidx, int Kp, int N,
+                    int32_t* __restrict__ rowmap, int* __restrict__ count) {
+  __shared__ int s_cnt[kCompactThreads];
+  const int t = threadIdx.x;
+  const int per = (N + kCompactThreads - 1) / kCompactThreads;
+  const int b = t * per;
+  const int e = (b + per < N) ? b + per : N;
+  auto keep = [&](int n) {
+    return (mask == nullptr || mask[n] != 0.f) && tidx[(size_t)n * Kp] != kSentinel;
+  };
+  int c = 0;
+  for (int n = b; n < e; ++n) c += keep(n) ? 1 : 0;
+  s_cnt[t] = c;
+  __syncthreads();
+  for (int off = 1; off < kCompactThreads; off <<= 1) {
+    const int v = t >= off ? s_cnt[t - off] : 0;
+    __syncthreads();
+    s_cnt[t] += v;
+    __syncthreads();
+  }
+  int o = s_cnt[t] - c;
+  for (int n = b; n < e; ++n)
+    if (keep(n)) rowmap[o++] = n;
+  if (t == kCompactThreads - 1) *count = s_cnt[t];
+}
+
+// Rows [row0, row0 + C) of the compacted token list: dst[r] = src[rowmap[row0 + r]]
+// (16-byte vectors, d8 per row) for the rows below *count, zeros past it.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4* __restrict__ src, int d8, const int32_t* __restrict__ rowmap,
+                   const int* __restrict__ count, int row0, int C, uint4* __restrict__ dst) {
+  const int live = *count;
+  const size_t total = (size_t)C * d8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / d8);
+    const int j = (int)(i - (size_t)r * d8);
+    const int q = row0 + r;
+    dst[i] = q < live ? src[(size_t)rowmap[q] * d8 + j] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The inverse for the rows below *count: dst[rowmap[row0 + r]] = src[r].
+__global__ void __launch_bounds__(256)
+scatter_rows_kernel(const uint4* __restrict__ src, int d8, const int32_t* __restrict__ rowmap,
+                    const int* __restrict__ count, int row0, int C, uint4* __restrict__ dst) {
+  const int live = *count;
+  int rows = live - row0;
+  rows = rows < 0 ? 0 : (rows > C ? C : rows);
+  const size_t total = (size_t)rows * d8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / d8);
+    const int j = (int)(i - (size_t)r * d8);
+    dst[(size_t)rowmap[row0 + r] * d8 + j] = src[i];
+  }
+}
+
 // Single block.  Sums block partials in a fixed order (deterministic).
 //  mode 0: *loss = sum(term_part) / sum(mask_part), or 0 if the mask sums to 0.
 //  mode 1: *cscale = g / sum(mask_part) (g = *grad or 1), or 0.

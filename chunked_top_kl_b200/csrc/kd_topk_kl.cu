@@ -36,12 +36,13 @@ struct Layout {
   int64_t n_prep_blocks = 0, n_merge_blocks = 0;
   size_t off_status = 0, off_scal = 0, off_mask_part = 0, off_term_part = 0;
   size_t off_tidx = 0, off_tp = 0, off_ent = 0, off_pm = 0, off_ps = 0, off_pg = 0, off_dz = 0;
+  size_t off_rowmap = 0, off_nrows = 0, off_hc = 0, off_dhc = 0;
   size_t total = 0;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-Layout make_layout(int64_t N, int64_t V, int64_t K, int64_t chunk) {
+Layout make_layout(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   Layout L;
   L.Kp = (int)round_up(K + 1, 4);
   L.ldz = round_up(V, 8);
@@ -61,6 +62,12 @@ Layout make_layout(int64_t N, int64_t V, int64_t K, int64_t chunk) {
   L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_dz = take(2 * (size_t)L.C * L.ldz);   // one dZ chunk (bf16)
+  // skipping rows with zero dZ: the kept tokens in order, their count, and
+  // one chunk of their H rows and of their dH rows (bf16)
+  L.off_rowmap = take(sizeof(int32_t) * (size_t)N);
+  L.off_nrows = take(sizeof(int));
+  L.off_hc = take(2 * (size_t)L.C * d);
+  L.off_dhc = take(2 * (size_t)L.C * d);
   L.total = o;
   return L;
 }
@@ -177,10 +184,11 @@ cudaError_t launch_gemm(int slot, int dev, int groups, const CUtensorMap& ta0, c
 template <class P0>
 cudaError_t launch_one(int slot, int dev, int groups, const CUtensorMap& ta, const CUtensorMap& tb,
                        const CUtensorMap& to, const ProbArgs& pa, Status* status,
-                       const typename P0::Epi::Params& ep, cudaStream_t s) {
+                       const typename P0::Epi::Params& ep, cudaStream_t s, DynRows dyn = DynRows{}) {
   GemmArgs a{};
   a.prob[0] = pa;
   a.status = status;
+  a.dyn = dyn;
   EpiNone::Params none{};
   return launch_gemm<P0, NoProb, kPair>(slot, dev, groups, ta, tb, to, ta, tb, to, a, ep, none, s);
 }
@@ -241,12 +249,13 @@ struct Variant {
   int logit_bf16;
   float T;
   float zscale, tfac, gfac;
+  bool skip_rows;       // backward over the tokens with a non-zero dZ row only
 };
 
 int make_variant(const kd_topk_kl_options* o, const void* logit, float T, Variant* v) {
   kd_topk_kl_options d{};
   if (o) d = *o;
-  if ((d.logit_bf16 | d.student_temperature) & ~1) return KD_ERR_INVALID_ARG;
+  if ((d.logit_bf16 | d.student_temperature | d.skip_masked_rows) & ~1) return KD_ERR_INVALID_ARG;
   for (int32_t r : d.reserved)
     if (r) return KD_ERR_INVALID_ARG;
   v->logit = logit;
@@ -255,6 +264,7 @@ int make_variant(const kd_topk_kl_options* o, const void* logit, float T, Varian
   v->zscale = d.student_temperature ? 1.0f / T : 1.0f;
   v->tfac = d.student_temperature ? T * T : 1.0f;
   v->gfac = d.student_temperature ? T : 1.0f;
+  v->skip_rows = d.skip_masked_rows != 0;
   return KD_OK;
 }
 
@@ -268,7 +278,7 @@ int common_checks(const void* H, const void* W, const int32_t* idx, const Varian
   if (!aligned(W, 16) || (H && !aligned(H, 16)) || !aligned(ws, 256)) return KD_ERR_INVALID_ARG;
   if ((idx && !aligned(idx, 4)) || (var.logit && !aligned(var.logit, var.logit_bf16 ? 2 : 4)))
     return KD_ERR_INVALID_ARG;
-  *L = make_layout(N, V, K, chunk);
+  *L = make_layout(N, d, V, K, chunk);
   if (ws_bytes < L->total) return KD_ERR_WORKSPACE;
   return KD_OK;
 }
@@ -314,7 +324,7 @@ const char* kd_status_string(int s) {
 
 size_t kd_topk_kl_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   if (check_shapes(N, d, V, K, 1.0f, chunk) != KD_OK) return 0;
-  return make_layout(N, V, K, chunk).total;
+  return make_layout(N, d, V, K, chunk).total;
 }
 
 int kd_topk_kl_forward(const void* H, const void* W, const int32_t* topk_idx,
@@ -419,6 +429,12 @@ int backward_checks(int64_t N, const float* lse, const float* grad_loss, const f
 // words are cleared and the teacher cache is prepared here; without it the
 // forward pass of the same call has done both.  Then the gradient scale and,
 // per chunk, the dZ recompute and the joint dH / dW launch.
+//
+// With var.skip_rows the chunks run over the compacted list of tokens whose
+// dZ row can be non-zero (mask != 0, teacher entries present), built on the
+// device: dH is cleared, and per chunk the kept tokens' H rows are gathered,
+// the GEMMs read the live row count from the device (chunks past it do no
+// work) and the chunk's dH rows are scattered back.
 int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const Variant& var,
                    const float* mask, int64_t N, int64_t d, int64_t V, int64_t K,
                    int64_t chunk, const Layout& L, const float* lse, const float* grad_loss,
@@ -440,6 +456,11 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
   double* mask_part = at<double>(workspace, L.off_mask_part);
   float* cscale = at<float>(workspace, L.off_scal);
   __nv_bfloat16* dz = at<__nv_bfloat16>(workspace, L.off_dz);
+  const bool compact = var.skip_rows;
+  int32_t* rowmap = at<int32_t>(workspace, L.off_rowmap);
+  int* nrows = at<int>(workspace, L.off_nrows);
+  __nv_bfloat16* hc = at<__nv_bfloat16>(workspace, L.off_hc);
+  __nv_bfloat16* dhc = at<__nv_bfloat16>(workspace, L.off_dhc);
 
   if (run_prep) {
     if (!evs.mark()) return KD_ERR_CUDA;
@@ -450,13 +471,25 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
   if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, nullptr, 0, 1, grad_loss, cscale);
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  if (compact) {
+    if (cudaMemsetAsync(dH, 0, sizeof(__nv_bfloat16) * (size_t)N * d, s) != cudaSuccess) return KD_ERR_CUDA;
+    if (!evs.mark()) return KD_ERR_CUDA;
+    compact_rows_kernel<<<1, kCompactThreads, 0, s>>>(mask, tidx, L.Kp, (int)N, rowmap, nrows);
+    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  }
 
+  // H as the recompute's A (K-major) and as the dW GEMM's B (MN-major), and
+  // the dH target: the caller's arrays, or one chunk of gathered rows
+  const void* hsrc = compact ? static_cast<const void*>(hc) : H;
+  void* dhdst = compact ? static_cast<void*>(dhc) : dH;
+  const int64_t hrows = compact ? L.C : N;
   CUtensorMap tmHk, tmWk, tmWmn, tmHmn, tmDH, tmDW;
-  if (!make_map(&tmHk, H, d, N, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, GeoP::B_ROWS) ||
-      !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, H, d, N, d, 64, BK) ||
-      !make_map(&tmDH, dH, d, N, d, 64, BM) || !make_map(&tmDW, dW, d, V, d, 32, BM, true))
+  if (!make_map(&tmHk, hsrc, d, hrows, d, BK, BM) || !make_map(&tmWk, W, d, V, d, BK, GeoP::B_ROWS) ||
+      !make_map(&tmWmn, W, d, V, d, 64, BK) || !make_map(&tmHmn, hsrc, d, hrows, d, 64, BK) ||
+      !make_map(&tmDH, dhdst, d, hrows, d, 64, BM) || !make_map(&tmDW, dW, d, V, d, 32, BM, true))
     return KD_ERR_CUDA;
   const int groups = resident_groups(dev);
+  const unsigned copy_blocks = (unsigned)(device_sms(dev) * 8);
 
   for (int64_t c0 = 0; c0 < N; c0 += chunk) {
     const int64_t Cc = (N - c0 < chunk) ? (N - c0) : chunk;
@@ -466,12 +499,24 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     if (!make_map(&tmZk, dz, L.ldz, Cc, L.ldz, BK, BM) || !make_map(&tmZmn, dz, L.ldz, Cc, L.ldz, 64, BK))
       return KD_ERR_CUDA;
 
+    const DynRows dyn = compact ? DynRows{nrows, (int)c0, (int)Cc} : DynRows{};
+    const int hrow0 = compact ? 0 : (int)c0;
+    if (compact) {
+      if (!evs.mark()) return KD_ERR_CUDA;
+      gather_rows_kernel<<<copy_blocks, 256, 0, s>>>(static_cast<const uint4*>(H), (int)(d / 8), rowmap, nrows,
+                                                    (int)c0, (int)Cc, reinterpret_cast<uint4*>(hc));
+      if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+    }
+
     // dZ for the chunk: recompute z = H W^T tile by tile.
     ProbArgs a3{};
     a3.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), true);
     a3.num_kb = (int)ceil_div(d, BK);
-    a3.a_row0 = (int)c0;
+    a3.a_row0 = hrow0;
+    a3.dyn_role = 1;
+    a3.dyn_bands_fastest = 1;
     EpiDz::Params e3{};
+    e3.rowmap = compact ? rowmap : nullptr;
     e3.rows_valid = (int)Cc;
     e3.row0 = (int)c0;
     e3.V = (int)V;
@@ -485,7 +530,8 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     e3.mask = mask;
     e3.cscale = cscale;
     if (!evs.mark()) return KD_ERR_CUDA;
-    if (launch_one<ProbDz>(1, dev, grid_for(a3.raster, groups), tmHk, tmWk, tmZk, a3, status, e3, s) != cudaSuccess)
+    if (launch_one<ProbDz>(1, dev, grid_for(a3.raster, groups), tmHk, tmWk, tmZk, a3, status, e3, s, dyn) !=
+        cudaSuccess)
       return KD_ERR_CUDA;
 
     // One launch for both gradient products of the chunk:
@@ -494,19 +540,29 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     //   problem 1: dW (+)= dZ^T H[chunk] (many short tiles, K = chunk)
     GemmArgs a45{};
     a45.status = status;
+    a45.dyn = dyn;
     a45.prob[0].raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), false);
     a45.prob[0].num_kb = (int)ceil_div(V, BK);
+    a45.prob[0].dyn_role = 1;
     a45.prob[1].raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
     a45.prob[1].num_kb = (int)ceil_div(Cc, BK);
-    a45.prob[1].b_k0 = (int)c0;
+    a45.prob[1].b_k0 = hrow0;
+    a45.prob[1].dyn_role = 2;
     plan_second_problem(a45, groups);
     EpiDh::Params e4{};
-    e4.row0 = (int)c0;
+    e4.row0 = hrow0;
     EpiDw::Params e5{};
     e5.accumulate = (accumulate_dW || c0 > 0) ? 1 : 0;
+    a45.prob[1].dyn_zero_fill = e5.accumulate ? 0 : 1;    // dW must be written even with no live row
     if (!evs.mark()) return KD_ERR_CUDA;
     if (launch_gemm<ProbDh, ProbDw, kPair>(2, dev, groups, tmZk, tmWmn, tmDH, tmZmn, tmHmn, tmDW, a45, e4, e5, s) != cudaSuccess)
       return KD_ERR_CUDA;
+    if (compact) {
+      if (!evs.mark()) return KD_ERR_CUDA;
+      scatter_rows_kernel<<<copy_blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(dhc), (int)(d / 8), rowmap,
+                                                     nrows, (int)c0, (int)Cc, static_cast<uint4*>(dH));
+      if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+    }
   }
   return KD_OK;
 }
@@ -550,7 +606,7 @@ int kd_topk_kl_backward_ex(const void* H, const void* W, const int32_t* topk_idx
   st = common_checks(H, W, topk_idx, var, N, d, V, K, chunk, workspace, workspace_bytes, &L);
   if (st != KD_OK) return st;
   if ((st = backward_checks(N, lse, grad_loss, mask, dH, dW)) != KD_OK) return st;
-  const int64_t launches = N > 0 ? 2 + 2 * ceil_div(N, chunk) : 0;
+  const int64_t launches = N > 0 ? (var.skip_rows ? 3 + 4 * ceil_div(N, chunk) : 2 + 2 * ceil_div(N, chunk)) : 0;
   if (events && n_events < launches + 1) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
@@ -586,7 +642,7 @@ int kd_topk_kl_forward_backward_ex(const void* H, const void* W, const int32_t* 
   if (st != KD_OK) return st;
   if (!loss || (N > 0 && !lse)) return KD_ERR_INVALID_ARG;
   if ((st = backward_checks(N, lse, grad_loss, mask, dH, dW)) != KD_OK) return st;
-  const int64_t launches = N > 0 ? 5 + 2 * ceil_div(N, chunk) : 0;
+  const int64_t launches = N > 0 ? (var.skip_rows ? 6 + 4 * ceil_div(N, chunk) : 5 + 2 * ceil_div(N, chunk)) : 0;
   if (events && n_events < launches + 1) return KD_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   LaunchEvents evs{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)), n_events, 0, s};
@@ -642,7 +698,7 @@ extern "C" int kd_topk_kl_forward_noalloc(const void* H, const void* W, const in
   // The forward pass needs no dZ chunk, so the smallest chunk keeps the
   // layout (and the size limit) to the prepared teacher cache, the per-token
   // partial log-sum-exp state and the status words.
-  if (make_layout(N, V, K, 1).total > kNoAllocScratchBytes) return KD_ERR_WORKSPACE;
+  if (make_layout(N, d, V, K, 1).total > kNoAllocScratchBytes) return KD_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KD_ERR_UNSUPPORTED;

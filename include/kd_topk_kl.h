@@ -32,7 +32,7 @@
  * scatter(p) with P = sum_k p = 0); its mask still counts in sum m.
  *
  * Variants selected through kd_topk_kl_options (the *_ex entry points; the
- * pages describe neither):
+ * pages describe none of them; skip_masked_rows changes only the work done):
  *  - logit_bf16: topk_logit holds bf16 values instead of fp32.
  *  - student_temperature: the usual distillation temperature on both sides:
  *      lse[n]  = log sum_v exp(z[n,v] / T)
@@ -92,8 +92,10 @@ const char* kd_status_string(int status);
  * need for these sizes (the same workspace size serves both).  Returns 0
  * for sizes that the entry points would reject.  It holds the prepared
  * teacher cache (sorted indices and probabilities, N x (K+1..K+4) x 8 B),
- * per-token partial log-sum-exp state, and one chunk of dZ
- * (chunk x round_up(V, 8) bf16): linear in N, and in chunk x V. */
+ * per-token partial log-sum-exp state, one chunk of dZ
+ * (chunk x round_up(V, 8) bf16), and for skip_masked_rows a token list
+ * (4 B per token) and two chunk x d bf16 row buffers: linear in N, and in
+ * chunk x V. */
 size_t kd_topk_kl_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk);
 
 /* Forward pass.  Writes *loss (device fp32 scalar) and lse[N] (device fp32;
@@ -196,7 +198,15 @@ int kd_topk_kl_forward_noalloc(const void* H, const void* W,
 typedef struct kd_topk_kl_options {
   int32_t logit_bf16;           /* 1: topk_logit is bf16 [N][K] (2-byte aligned) */
   int32_t student_temperature;  /* 1: student logits divided by T too, term times T^2 */
-  int32_t reserved[6];
+  int32_t skip_masked_rows;     /* 1: the backward pass works on the tokens whose dZ row can be
+                                   non-zero only (mask != 0 and teacher entries present): they are
+                                   listed on the device and processed chunk by chunk, rows of the
+                                   others are skipped (their dH rows are written as 0).  Same
+                                   results except for the fp32 summation order of dW.  Launches
+                                   (for events): backward 3 + 4 * ceil(N / chunk), fused
+                                   6 + 4 * ceil(N / chunk) (a compaction kernel, and per chunk a
+                                   row gather and a dH row scatter around the two GEMMs). */
+  int32_t reserved[5];
 } kd_topk_kl_options;
 
 /* kd_topk_kl_forward with options; topk_logit is fp32 or bf16 as

@@ -49,6 +49,7 @@ def test_launch_count_and_config_block():
     assert bench.launches_per_step(32768, 4096) == 5 + 2 * 8
     assert bench.launches_per_step(300, 128) == 5 + 2 * 3
     assert bench.launches_per_step(0, 128) == 0
+    assert bench.launches_per_step(32768, 4096, skip_rows=True) == 6 + 4 * 8
     blk = bench.config_block(workloads.get_config(3), 4)
     assert blk["global_batch"] == 4 * 32768 and blk["workload"].startswith("gptoss_head")
 

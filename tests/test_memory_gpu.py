@@ -7,7 +7,8 @@ For the long-context sweep's shape (d = 2048, V = 128256, K = 100, chunk
 measured at N = 4K ... 256K tokens, fitted by least squares, and compared
 with the analytic per-token bytes:
   H and dH (2 x 2d), teacher cache (8K), mask and lse (8), prepared teacher
-  (8 Kp + 4), forward partials (16 splits x 12) and per-block sums.
+  (8 Kp + 4), forward partials (16 splits x 12), the kept-token list for
+  skipping masked rows (4) and per-block sums.
 """
 
 import numpy as np
@@ -58,7 +59,7 @@ def test_peak_memory_linear_in_tokens(kd):
     slope, icpt = np.polyfit(Ns, peaks, 1)
     resid = np.abs(peaks - (slope * Ns + icpt)) / peaks
     Kp = ((K + 1 + 3) // 4) * 4
-    per_token = 2 * 2 * D + 8 * K + 8 + 8 * Kp + 4 + 16 * 12
+    per_token = 2 * 2 * D + 8 * K + 8 + 8 * Kp + 4 + 16 * 12 + 4
     print("peaks GiB", peaks / 2**30, "slope B/token", slope, "analytic", per_token)
     assert resid.max() < 0.03, resid
     assert abs(slope - per_token) <= 0.10 * per_token, (slope, per_token)

@@ -3,7 +3,9 @@ pages) against the fp64 oracle, through the C ABI's *_ex entry points:
 
 * empty teacher slots (index -1), including tokens with no entry at all;
 * a bf16 teacher cache (topk_logit in bf16);
-* the student at temperature T with the T^2 factor.
+* the student at temperature T with the T^2 factor;
+* skipping the rows of masked tokens in the backward pass (the same loss
+  and gradients, less work).
 
 Same tolerances as the main parity tests: loss relative error <= 1e-3,
 lse absolute error <= 2e-3, relative Frobenius error <= 1e-2 for dH, dW.
@@ -146,3 +148,57 @@ def test_variants_combined_fused(kd):
         assert torch.equal(a[k], b[k]), k
     ref = _oracle(x, 1.5, grad=0.6, student_T=True)
     _assert_parity(a, ref, "combined")
+
+
+def _masked_inputs(N, d, V, K, seed, frac):
+    x = _inputs(N, d, V, K, seed=seed, mask="ones")
+    g = torch.Generator().manual_seed(900 + seed)
+    x["mask"] = (torch.rand(N, generator=g) >= frac).float()
+    return x
+
+
+@pytest.mark.parametrize("frac,chunk", [(0.05, 128), (0.6, 64), (1.0, 96)], ids=["drop5", "drop60", "all"])
+def test_skip_masked_rows(kd, frac, chunk):
+    # the backward over the kept tokens only: the forward is untouched, dH
+    # equal bit for bit (every dZ row is computed the same way), dW equal up
+    # to the fp32 order of the chunk sums; with 60 % dropped the trailing
+    # chunks have no live row, with everything dropped dW must still be zeroed
+    x = _masked_inputs(700, 136, 3000, 24, seed=44, frac=frac)
+    x["topk_idx"] = _empty_slots(x["topk_idx"], 44, frac=0.1, empty_rows=(3,))
+    a = _run(kd, x, 1.0, chunk, grad=1.4, student_temperature=False)
+    g = {k: v.cuda() for k, v in x.items()}
+    ws = kd.alloc_workspace(700, 136, 3000, 24, chunk, "cuda")
+    dW = torch.full((3000, 136), float("nan"), device="cuda")     # overwritten, never read
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(kd.forward_backward_launches(700, chunk, True) + 1)]
+    for e in evs:
+        e.record()                       # creates the CUDA event behind each object
+    loss, lse, dH, dW = kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, chunk,
+                                            grad_loss=torch.tensor(1.4, device="cuda"), dW=dW, workspace=ws,
+                                            events=evs, skip_masked_rows=True)
+    st, nbad = kd.check(ws)
+    assert st == 0 and nbad == 0
+    b = {"loss": float(loss.item()), "lse": lse.cpu(), "dH": dH.cpu(), "dW": dW.cpu()}
+    assert a["loss"] == b["loss"] and torch.equal(a["lse"], b["lse"])
+    assert torch.equal(a["dH"], b["dH"])
+    assert torch.isfinite(b["dW"]).all()
+    if frac < 1.0:
+        assert _rfro(b["dW"].double().numpy(), a["dW"].double().numpy()) <= 1e-5
+        _assert_parity(b, _oracle(x, 1.0, grad=1.4), "skip rows")
+    else:
+        assert torch.count_nonzero(b["dW"]) == 0 and torch.count_nonzero(b["dH"]) == 0
+    for e in evs:
+        e.synchronize()
+
+
+def test_skip_masked_rows_accumulates(kd):
+    x = _masked_inputs(500, 64, 2000, 16, seed=45, frac=0.3)
+    g = {k: v.cuda() for k, v in x.items()}
+    ws = kd.alloc_workspace(500, 64, 2000, 16, 128, "cuda")
+    loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 128, workspace=ws)
+    base = torch.randn(2000, 64, device="cuda") * 1e-4       # the gradient's scale: no cancellation
+    dW = base.clone()
+    dH, dW = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 128, lse, dW=dW,
+                         accumulate_dW=True, workspace=ws, skip_masked_rows=True)
+    _, ref = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 128, lse, workspace=ws)
+    assert kd.check(ws)[0] == 0
+    assert _rfro((dW - base).double().cpu().numpy(), ref.double().cpu().numpy()) <= 1e-5
