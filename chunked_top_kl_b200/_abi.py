@@ -32,6 +32,8 @@ EXPORTS = (
     "kd_topk_kl_forward_ex",
     "kd_topk_kl_backward_ex",
     "kd_topk_kl_forward_backward_ex",
+    "kd_teacher_topk_workspace_size",
+    "kd_teacher_topk",
 )
 
 
@@ -91,6 +93,10 @@ def load() -> ctypes.CDLL:
         lib.kd_topk_kl_forward_backward_ex.argtypes = [p, p, p, p, p, i64, i64, i64, i64, f32, i64, p, p, p,
                                                        p, p, i32, p, sz, p, evp, i64, opt]
         lib.kd_topk_kl_forward_backward_ex.restype = i32
+        lib.kd_teacher_topk_workspace_size.argtypes = [i64, i64, i64, i64, i64]
+        lib.kd_teacher_topk_workspace_size.restype = sz
+        lib.kd_teacher_topk.argtypes = [p, p, i64, i64, i64, i64, i64, p, p, p, sz, p]
+        lib.kd_teacher_topk.restype = i32
         _lib = lib
     return _lib
 
@@ -195,3 +201,12 @@ def kd_topk_kl_forward_backward_ex(H, W, topk_idx, topk_logit, mask, N, d, V, K,
                                                      chunk, loss, lse, grad_loss, dH, dW,
                                                      int(accumulate_dW), workspace, workspace_bytes,
                                                      stream, arr, n, _opt(options)))
+
+
+def kd_teacher_topk_workspace_size(N: int, d: int, V: int, K: int, chunk: int) -> int:
+    return int(load().kd_teacher_topk_workspace_size(N, d, V, K, chunk))
+
+
+def kd_teacher_topk(Ht, Wt, N, d, V, K, chunk, topk_idx, topk_logit, workspace, workspace_bytes, stream) -> int:
+    return int(load().kd_teacher_topk(Ht, Wt, N, d, V, K, chunk, topk_idx, topk_logit, workspace,
+                                      workspace_bytes, stream))

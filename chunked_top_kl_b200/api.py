@@ -192,6 +192,32 @@ def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chun
     return loss, lse, dH, dW
 
 
+def teacher_topk(Ht, Wt, K: int, chunk: int = 1024,
+                 workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The teacher top-K cache of hidden states Ht [N,d] under head Wt [V,d]
+    (both bf16): returns (topk_idx [N,K] int32, topk_logit [N,K] fp32), each
+    row's K largest logits largest first, ties in increasing column order."""
+    if not (Ht.is_cuda and Wt.is_cuda) or Ht.dtype != torch.bfloat16 or Wt.dtype != torch.bfloat16:
+        raise TypeError("teacher_topk: Ht and Wt must be bfloat16 CUDA tensors")
+    if not (Ht.is_contiguous() and Wt.is_contiguous()) or Ht.shape[1] != Wt.shape[1]:
+        raise ValueError("teacher_topk: contiguous Ht [N,d] and Wt [V,d] expected")
+    N, d = Ht.shape
+    V = Wt.shape[0]
+    dev = Ht.device
+    if workspace is None:
+        n = _abi.kd_teacher_topk_workspace_size(N, d, V, K, chunk)
+        if n == 0:
+            raise ValueError("teacher_topk: unsupported sizes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    idx = torch.empty((N, K), dtype=torch.int32, device=dev)
+    val = torch.empty((N, K), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = _abi.kd_teacher_topk(_ptr(Ht), _ptr(Wt), N, d, V, int(K), int(chunk), _ptr(idx), _ptr(val),
+                              _ptr(workspace), workspace.numel(), stream)
+    _raise(st, "kd_teacher_topk")
+    return idx, val
+
+
 def check(workspace: torch.Tensor) -> Tuple[int, int]:
     """Synchronise the current stream and read the device status words:
     returns (status, bad_index_count)."""

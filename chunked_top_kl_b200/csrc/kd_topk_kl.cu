@@ -20,6 +20,7 @@
 #include "../../include/kd_topk_kl.h"
 #include "kd_gemm.cuh"
 #include "kd_small_kernels.cuh"
+#include "kd_topk_select.cuh"
 
 using namespace kd;
 
@@ -240,6 +241,7 @@ using ProbFwd = Prob<EpiFwd, false, false, kL2EvictLast, kL2Normal>;  // A = H (
 using ProbDz = Prob<EpiDz, false, false, kL2EvictLast, kL2Normal>;    // A = H chunk, B = W
 using ProbDh = Prob<EpiDh, false, true>;      // A = dZ (K-major over V), B = W (MN-major over d)
 using ProbDw = Prob<EpiDw, true, true, kL2Normal, kL2EvictLast>;      // A = dZ^T (MN-major over V), B = H chunk
+using ProbZ32 = Prob<EpiDw, false, false, kL2EvictLast, kL2Normal>;   // teacher logits, fp32 store: A = Ht, B = Wt
 
 // The loss as one call computes it: the teacher logits and their type, T,
 // and the factors of the student-temperature variant (zs on the student
@@ -662,6 +664,94 @@ int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_cou
   if (bad_index_count) *bad_index_count = (int64_t)h.bad_index;
   if (h.timeout) return KD_ERR_TIMEOUT;
   if (h.bad_index) return KD_ERR_BAD_INDEX;
+  return KD_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- teacher top-K cache writer
+//
+// The offline cache the loss consumes: for each position, the K largest
+// logits of the teacher head and their indices (blog post, "Two systems
+// changes", offline distillation paragraph).  Per chunk of tokens, the
+// teacher logits z = Ht Wt^T are computed by the same tcgen05 GEMM as the
+// loss (fp32 tiles stored through TMA into a chunk buffer) and each row's
+// top K are selected exactly (topk_select_kernel).
+
+namespace {
+
+// Status words first (as in the loss workspace, so kd_topk_kl_check reads
+// them), then one chunk of fp32 logits.
+struct TopkLayout {
+  int64_t C = 0, ldz = 0;
+  size_t off_status = 0, off_z = 0, total = 0;
+};
+
+TopkLayout make_topk_layout(int64_t N, int64_t V, int64_t chunk) {
+  TopkLayout L;
+  L.C = N > 0 ? (chunk < N ? chunk : N) : 1;
+  L.ldz = round_up(V, 4);
+  L.off_status = 0;
+  L.off_z = align256(sizeof(Status));
+  L.total = L.off_z + align256(sizeof(float) * (size_t)L.C * L.ldz);
+  return L;
+}
+
+int topk_checks(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
+  if (N < 0 || d <= 0 || V <= 0 || K <= 0 || chunk <= 0) return KD_ERR_INVALID_ARG;
+  if (d % 8 != 0 || K > kMaxTopK || K > V) return KD_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) || V >= (int64_t(1) << 31) || d >= (int64_t(1) << 24)) return KD_ERR_UNSUPPORTED;
+  return KD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kd_teacher_topk_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
+  if (topk_checks(N, d, V, K, chunk) != KD_OK) return 0;
+  return make_topk_layout(N, V, chunk).total;
+}
+
+int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_t V, int64_t K,
+                    int64_t chunk, int32_t* topk_idx, float* topk_logit, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int st = topk_checks(N, d, V, K, chunk);
+  if (st != KD_OK) return st;
+  if (!Wt || !workspace || (N > 0 && (!Ht || !topk_idx || !topk_logit))) return KD_ERR_INVALID_ARG;
+  if (!aligned(Wt, 16) || (Ht && !aligned(Ht, 16)) || !aligned(workspace, 256) ||
+      (topk_idx && !aligned(topk_idx, 4)) || (topk_logit && !aligned(topk_logit, 4)))
+    return KD_ERR_INVALID_ARG;
+  const TopkLayout L = make_topk_layout(N, V, chunk);
+  if (workspace_bytes < L.total) return KD_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Status* status = at<Status>(workspace, L.off_status);
+  if (cudaMemsetAsync(status, 0, sizeof(Status), s) != cudaSuccess) return KD_ERR_CUDA;
+  if (N == 0) return KD_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
+  float* zbuf = at<float>(workspace, L.off_z);
+
+  CUtensorMap tmH, tmW;
+  if (!make_map(&tmH, Ht, d, N, d, BK, BM) || !make_map(&tmW, Wt, d, V, d, BK, GeoP::B_ROWS)) return KD_ERR_CUDA;
+  const int groups = resident_groups(dev);
+  for (int64_t c0 = 0; c0 < N; c0 += chunk) {
+    const int64_t Cc = (N - c0 < chunk) ? (N - c0) : chunk;
+    // fp32 logits of the chunk: [Cc][ldz], columns >= V never written (TMA clips them)
+    CUtensorMap tmZ;
+    if (!make_map(&tmZ, zbuf, V, Cc, L.ldz, 32, BM, true)) return KD_ERR_CUDA;
+    ProbArgs a{};
+    a.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), true);
+    a.num_kb = (int)ceil_div(d, BK);
+    a.a_row0 = (int)c0;
+    EpiDw::Params e{};
+    e.accumulate = 0;
+    if (launch_one<ProbZ32>(3, dev, grid_for(a.raster, groups), tmH, tmW, tmZ, a, status, e, s) != cudaSuccess)
+      return KD_ERR_CUDA;
+    topk_select_kernel<<<(unsigned)Cc, kSelectThreads, 0, s>>>(zbuf, L.ldz, (int)V, (int)K, (int)c0, topk_idx,
+                                                               topk_logit);
+    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  }
   return KD_OK;
 }
 

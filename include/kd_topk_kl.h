@@ -243,6 +243,23 @@ int kd_topk_kl_forward_backward_ex(const void* H, const void* W,
                                    void* const* events, int64_t n_events,
                                    const kd_topk_kl_options* options);
 
+/* Teacher top-K cache writer: the offline cache that the loss consumes (blog
+ * post, "Two systems changes", offline distillation paragraph: the teacher's
+ * top-K logits stored per position).  For teacher hidden states Ht bf16
+ * [N][d] and teacher head Wt bf16 [V][d] it writes, per token, the K largest
+ * logits z = Ht Wt^T (fp32 accumulation of the bf16 products) and their
+ * column indices, largest first, equal logits in increasing column order:
+ * topk_idx int32 [N][K], topk_logit fp32 [N][K] (device, caller-owned).
+ * Tokens are processed `chunk` at a time: the logits of one chunk are stored
+ * in the workspace (chunk x round_up(V, 4) fp32) and each row's top K is
+ * selected exactly.  Supported: 1 <= K <= min(V, 512), d % 8 == 0; Ht and Wt
+ * 16-byte aligned, the workspace 256-byte aligned.  kd_topk_kl_check on this
+ * workspace reports a pipeline timeout. */
+size_t kd_teacher_topk_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk);
+int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_t V, int64_t K,
+                    int64_t chunk, int32_t* topk_idx, float* topk_logit,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then reads the device-side status words that the
  * last forward or backward call on this workspace wrote.  Returns KD_OK,
  * KD_ERR_BAD_INDEX (teacher index outside [0, V) seen), KD_ERR_TIMEOUT (a
