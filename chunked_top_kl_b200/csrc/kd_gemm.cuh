@@ -62,7 +62,8 @@ struct ProbArgs {
   int num_kb;           // BK-wide K blocks per tile
   int a_row0, b_row0;   // added to the row (M / N) coordinate
   int a_k0, b_k0;       // added to the K coordinate
-  int dyn_role;         // with GemmArgs::dyn: 1 = the live rows are this GEMM's M, 2 = its K
+  int dyn_role;         // with GemmArgs::dyn: the live rows are this GEMM's M (1: one tile per
+                        // unit, 3: band x column range units) or its K (2)
   int dyn_bands_fastest;
   int dyn_zero_fill;    // role 2 with no live rows: still write the (zero) output tiles
 };
@@ -96,6 +97,8 @@ __device__ __forceinline__ void apply_live_rows(GemmArgs& a, int rows, int ngrou
     ProbArgs& pa = a.prob[p];
     if (pa.dyn_role == 1) {
       pa.raster = tile_raster(ceil_div64(rows, G::TILE_M), pa.raster.n_tiles, pa.dyn_bands_fastest != 0);
+    } else if (pa.dyn_role == 3) {
+      pa.raster = forward_raster(ceil_div64(rows, G::TILE_M), pa.raster.n_tiles, ngroups);
     } else if (pa.dyn_role == 2) {
       pa.num_kb = (int)ceil_div64(rows, BK);
       if (rows == 0 && !pa.dyn_zero_fill) pa.raster.num_units = 0;
@@ -171,9 +174,16 @@ struct EpiCtx {
 // Writes one 128-byte segment per thread (its row) into the next staging
 // buffer with the 128-byte swizzle, then one thread stores (or adds) the
 // 128-row box to global memory at (x, y) with TMA.
+struct NoFix {
+  __device__ __forceinline__ void operator()(uint32_t, uint32_t) const {}
+};
+
+// `fix(rowa, sw)` may rewrite elements of the thread's own row after it is
+// written (16-byte chunk k of the row sits at rowa + ((k ^ sw) << 4)).
+template <class Fix = NoFix>
 __device__ __forceinline__ void stage_store(EpiCtx& cx, const CUtensorMap* tm, int x, int y,
                                             const uint32_t (&w)[32], bool reduce_add,
-                                            int hint = kL2Normal) {
+                                            int hint = kL2Normal, const Fix& fix = Fix{}) {
   const uint32_t buf = cx.stage[cx.seq & 1u];
   if (cx.issuer && cx.seq >= 2) bulk_wait_read<1>();     // buffer's previous store has read it
   epilogue_bar_sync(128);
@@ -182,6 +192,7 @@ __device__ __forceinline__ void stage_store(EpiCtx& cx, const CUtensorMap* tm, i
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     st_shared_v4(rowa + (((uint32_t)k ^ sw) << 4), w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  fix(rowa, sw);
   fence_proxy_async_shared();
   epilogue_bar_sync(128);
   if (cx.issuer) {
@@ -364,7 +375,7 @@ __device__ __forceinline__ bool epi_unit(const Smem<G>& L, RoleState& st, uint32
   decode_unit(pa.raster, u, m, split, n0, n1);
   const int grow = m * G::TILE_M + row;
   cx.row_base = m * G::TILE_M + (int)rank * BM;
-  epi.begin_unit(ep, grow, split, n0);
+  epi.begin_unit(ep, grow, split, n0, cx);
   for (int n = n0; n < n1; ++n) {
     // One outcome for all 128 epilogue threads: tcgen05.ld needs whole
     // warps and the store path synchronises the four warps.
@@ -490,6 +501,59 @@ __device__ __forceinline__ int lower_bound_row(const int32_t* row, int len, int 
   return lo;
 }
 
+// v[i] for a run-time i in [0, 64), by a tree of selects on i's bits: the
+// array stays in registers (an indexed read would put it in local memory).
+__device__ __forceinline__ float pick64(const float (&v)[64], int i) {
+  float a[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) a[k] = (i & 32) ? v[k + 32] : v[k];
+#pragma unroll
+  for (int w = 16; w > 0; w >>= 1) {
+    const bool hi = (i & w) != 0;
+#pragma unroll
+    for (int k = 0; k < w; ++k) a[k] = hi ? a[k + w] : a[k];
+  }
+  return a[0];
+}
+
+// A thread's walk over its token's index-sorted teacher entries (row of Kp
+// slots ending in kSentinel) as the vocabulary columns stream past in
+// increasing order.  (i0, p0) is the next entry; the one after it is loaded
+// as soon as i0 is consumed, long before it is compared, so a hit does not
+// stall the epilogue on a global load.
+struct TeacherCursor {
+  const int32_t* trow;
+  const float* prow;
+  int cur, kp;
+  int i0, i1;
+  float p0, p1;
+
+  __device__ __forceinline__ void none() {
+    trow = nullptr;
+    prow = nullptr;
+    cur = kp = 0;
+    i0 = i1 = kSentinel;
+    p0 = p1 = 0.f;
+  }
+  __device__ __forceinline__ void start(const int32_t* t, const float* p, int kp_, int col) {
+    trow = t;
+    prow = p;
+    kp = kp_;
+    cur = lower_bound_row(t, kp_, col);
+    i0 = t[cur];
+    p0 = p[cur];
+    i1 = cur + 1 < kp ? t[cur + 1] : kSentinel;
+    p1 = cur + 1 < kp ? p[cur + 1] : 0.f;
+  }
+  __device__ __forceinline__ void advance() {
+    i0 = i1;
+    p0 = p1;
+    ++cur;
+    i1 = cur + 1 < kp ? trow[cur + 1] : kSentinel;
+    p1 = cur + 1 < kp ? prow[cur + 1] : 0.f;
+  }
+};
+
 // Forward: running max / sum-exp over the unit's vocabulary columns and the
 // gathered sum of p * z at the teacher's columns; one (m, s, g) partial per
 // token per split.  Columns >= V are -inf.  The sum is of exp((z - m) * zs)
@@ -506,25 +570,19 @@ struct EpiFwd {
     float* part_s;
     float* part_g;
   };
-  float mrun, srun, grun, np;
-  int cur, nidx, grow;
-  const int32_t* trow;
-  const float* prow;
+  float mrun, srun, grun;
+  int grow;
+  TeacherCursor tc;
 
-  __device__ __forceinline__ void begin_unit(const Params& P, int grow_, int, int n0) {
+  __device__ __forceinline__ void begin_unit(const Params& P, int grow_, int, int n0, const EpiCtx&) {
     grow = grow_;
     mrun = -INFINITY;
     srun = 0.f;
     grun = 0.f;
-    nidx = kSentinel;
-    np = 0.f;
-    if (grow < P.N) {
-      trow = P.tidx + (size_t)grow * P.Kp;
-      prow = P.tp + (size_t)grow * P.Kp;
-      cur = lower_bound_row(trow, P.Kp, n0 * BN);
-      nidx = trow[cur];
-      np = prow[cur];
-    }
+    if (grow < P.N)
+      tc.start(P.tidx + (size_t)grow * P.Kp, P.tp + (size_t)grow * P.Kp, P.Kp, n0 * BN);
+    else
+      tc.none();
   }
 
   __device__ __forceinline__ void tile(const Params& P, const CUtensorMap*, int, int n, uint32_t taddr,
@@ -540,16 +598,9 @@ struct EpiFwd {
         for (int i = 0; i < 64; ++i)
           if (c0 + i >= P.V) v[i] = -INFINITY;
       }
-      if (nidx < c0 + 64) {                 // a teacher column in this group (rare)
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          if (c0 + i == nidx) {
-            grun += np * v[i];
-            ++cur;
-            nidx = trow[cur];
-            np = prow[cur];
-          }
-        }
+      while (tc.i0 < c0 + 64) {             // a teacher column in this group (rare)
+        grun += tc.p0 * pick64(v, tc.i0 - c0);
+        tc.advance();
       }
       // group max (pairwise tree), then the rescaled running sum-exp with
       // 2^(z log2(e) - m log2(e)): one FFMA and one ex2 per element
@@ -600,7 +651,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // Backward, per chunk: dZ = c_n (exp(z zs - lse_n) - p at the teacher's
-// columns), rounded to bf16 and stored for the chunk's tokens (row-major,
+// columns), one unit per band and range of column tiles (the row's scale,
+// lse and teacher cursor set once per unit), rounded to bf16 and stored for
+// the chunk's tokens (row-major,
 // ldz columns) through shared memory and TMA (`out`: the chunk buffer, bf16,
 // box {64, 128}, 128-byte swizzle).  zs = 1, or 1 / T for the
 // student-temperature variant, whose extra factor T on c_n comes in as gfac.
@@ -622,35 +675,37 @@ struct EpiDz {
     const float* mask;     // may be null
     const float* cscale;   // device scalar g / sum(mask)
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
-  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
+  // The row's state for a unit (a band and a range of column tiles, in
+  // increasing order): c exp(z zs - lse) = 2^(z zl2 - bias) with
+  // bias = lse log2(e) - log2(c), one FFMA and one ex2 per element.  c = 0
+  // (masked token, token without teacher entries) and rows past the chunk
+  // give bias = +inf, hence exact zeros.  A negative c (negative upstream
+  // gradient or mask weight) is applied as a sign flip of the packed bf16
+  // pair.
+  float bias, c;
+  uint32_t sgn;
+  TeacherCursor tc;
 
-  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int r, int n,
-                                       uint32_t taddr, EpiCtx& cx) {
-    const bool valid = r < (cx.rows_valid >= 0 ? cx.rows_valid : P.rows_valid);
-    const int grow = valid && P.rowmap ? P.rowmap[P.row0 + r] : P.row0 + r;
-    // c exp(z zs - lse) = 2^(z zl2 - bias) with bias = lse log2(e) - log2(c):
-    // one FFMA and one ex2 per element.  c = 0 (masked token, token without
-    // teacher entries) and rows past the chunk give bias = +inf, hence exact
-    // zeros.  A negative c (negative upstream gradient or mask weight) is
-    // applied as a sign flip of the packed bf16 pair.
-    float bias = INFINITY, c = 0.f;
-    uint32_t sgn = 0u;
-    const int32_t* trow = nullptr;
-    const float* prow = nullptr;
-    int cur = 0, nidx = kSentinel;
-    float np = 0.f;
-    if (valid) {
-      trow = P.tidx + (size_t)grow * P.Kp;
-      prow = P.tp + (size_t)grow * P.Kp;
+  __device__ __forceinline__ void begin_unit(const Params& P, int r, int, int n0, const EpiCtx& cx) {
+    bias = INFINITY;
+    c = 0.f;
+    sgn = 0u;
+    tc.none();
+    if (r < (cx.rows_valid >= 0 ? cx.rows_valid : P.rows_valid)) {
+      const int grow = P.rowmap ? P.rowmap[P.row0 + r] : P.row0 + r;
+      const int32_t* trow = P.tidx + (size_t)grow * P.Kp;
+      const float* prow = P.tp + (size_t)grow * P.Kp;
+      tc.start(trow, prow, P.Kp, n0 * BN);
       const float cs = trow[0] == kSentinel ? 0.f : (P.mask ? P.mask[grow] : 1.f) * (*P.cscale) * P.gfac;
       c = fabsf(cs);
       sgn = cs < 0.f ? 0x80008000u : 0u;
       bias = P.lse[grow] * kLog2e - log2f(c);
-      cur = lower_bound_row(trow, P.Kp, n * BN);
-      nidx = trow[cur];
-      np = prow[cur];
     }
+  }
+  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
+
+  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int, int n,
+                                       uint32_t taddr, EpiCtx& cx) {
     const float zl2 = P.zl2;
 #pragma unroll 1
     for (int j = 0; j < BN / 64; ++j) {
@@ -665,17 +720,6 @@ struct EpiDz {
         v[i] = ex2_approx(e.x);
         v[i + 1] = ex2_approx(e.y);
       }
-      if (nidx < c0 + 64) {                 // a teacher column in this group (rare)
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          if (c0 + i == nidx) {
-            v[i] -= c * np;
-            ++cur;
-            nidx = trow[cur];
-            np = prow[cur];
-          }
-        }
-      }
       if (c0 + 64 > P.V) {                  // last vocabulary tile: zero columns >= V
 #pragma unroll
         for (int i = 0; i < 64; ++i)
@@ -688,7 +732,20 @@ struct EpiDz {
 #pragma unroll
         for (int i = 0; i < 32; ++i) w[i] ^= sgn;
       }
-      stage_store(cx, out, c0, cx.row_base, w, false);
+      // the teacher's columns in this group (rare): subtract c p from the
+      // staged bf16 value, stored as sign * c exp(..), so minus (signed c) p
+      const float cs = sgn ? -c : c;
+      TeacherCursor& t = tc;
+      stage_store(cx, out, c0, cx.row_base, w, false, kL2Normal, [&](uint32_t rowa, uint32_t sw) {
+        while (t.i0 < c0 + 64) {
+          const uint32_t off = (uint32_t)(t.i0 - c0);
+          const uint32_t a = rowa + (((off >> 3) ^ sw) << 4) + ((off & 7u) << 1);
+          const uint16_t h = ld_shared_u16(a);
+          const float x = __bfloat162float(__ushort_as_bfloat16(h)) - cs * t.p0;
+          st_shared_u16(a, __bfloat16_as_ushort(__float2bfloat16_rn(x)));
+          t.advance();
+        }
+      });
     }
   }
 };
@@ -701,7 +758,7 @@ struct EpiDh {
   struct Params {
     int row0;
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, const EpiCtx&) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
   __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int, int n,
@@ -727,7 +784,7 @@ struct EpiDw {
   struct Params {
     int accumulate;        // `out`: dW [V][d] fp32, box {32, 128}, 128-byte swizzle
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, const EpiCtx&) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 
   __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int, int n,
@@ -758,7 +815,7 @@ struct EpiNone {
   struct Params {
     int unused;
   };
-  __device__ __forceinline__ void begin_unit(const Params&, int, int, int) {}
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, const EpiCtx&) {}
   __device__ __forceinline__ void tile(const Params&, const CUtensorMap*, int, int, uint32_t, EpiCtx&) {}
   __device__ __forceinline__ void end_unit(const Params&, int, int) {}
 };

@@ -59,8 +59,9 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
   return r;
 }
 
-// Forward pass: a unit is a band and a range of vocabulary tiles whose
-// running log-sum-exp one CTA carries.  Picks the number of ranges
+// Forward pass (and the dZ recompute): a unit is a band and a range of
+// vocabulary tiles whose running log-sum-exp (or teacher-column cursor) one
+// CTA carries.  Picks the number of ranges
 // (<= kMaxSplits) minimising waves x longest range on `grid` CTAs; every
 // range is non-empty.
 //
@@ -69,10 +70,10 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
 // the same ranges side by side, group_m = grid / 2 (two ranges per wave),
 // capped so the group's A bands (band_bytes each, kept in L2) take at most
 // half of `l2_budget`, and evened out over the groups.
-inline Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid, int64_t band_bytes = 0,
-                             int64_t l2_budget = 0) {
+KD_HD Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid, int64_t band_bytes = 0,
+                            int64_t l2_budget = 0) {
   int best_s = 1;
-  int64_t best_cost = INT64_MAX;
+  int64_t best_cost = (int64_t)1 << 62;
   for (int s = 1; s <= kMaxSplits && s <= n_tiles; ++s) {
     const int64_t cost = ceil_div64(m_tiles * s, grid) * ceil_div64(n_tiles, s);
     if (cost < best_cost) { best_cost = cost; best_s = s; }

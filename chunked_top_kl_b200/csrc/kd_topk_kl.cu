@@ -511,12 +511,13 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     }
 
     // dZ for the chunk: recompute z = H W^T tile by tile.
+    // Units are a band and a range of column tiles, so each epilogue thread
+    // sets up its token (scale, lse, teacher cursor) once per unit.
     ProbArgs a3{};
-    a3.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), true);
+    a3.raster = forward_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), groups);
     a3.num_kb = (int)ceil_div(d, BK);
     a3.a_row0 = hrow0;
-    a3.dyn_role = 1;
-    a3.dyn_bands_fastest = 1;
+    a3.dyn_role = 3;
     EpiDz::Params e3{};
     e3.rowmap = compact ? rowmap : nullptr;
     e3.rows_valid = (int)Cc;
