@@ -87,7 +87,24 @@ struct GemmArgs {
   JointPlan joint;
   DynRows dyn;
   Status* status;
+  // Optional wave pacing of problem 0 (zeroed counters, one per wave): a
+  // CTA's producer starts its k-th unit only once every CTA with a k-th unit
+  // has issued all loads of its (k-1)-th, so the CTAs that share operand
+  // tiles in a wave keep reading them together.  Pacing only: a wait gives
+  // up after kWaveWaitNs and the CTA goes on.
+  unsigned int* wave_sync;
 };
+
+constexpr uint64_t kWaveWaitNs = 20000000ull;   // 20 ms
+
+__device__ __forceinline__ void wave_barrier(unsigned int* counter, unsigned int expected) {
+  atomicAdd(counter, 1u);
+  const uint64_t t0 = globaltimer_ns();
+  while (*reinterpret_cast<volatile unsigned int*>(counter) < expected) {
+    if (globaltimer_ns() - t0 > kWaveWaitNs) break;
+    __nanosleep(64);
+  }
+}
 
 // The schedule of a launch with live row count `rows` (see DynRows).
 template <class G, bool HAS_P1>
@@ -464,6 +481,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     if (lane == 0)
       failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap* tA,
                                   const CUtensorMap* tB, int u) {
+        if constexpr (std::is_same<decltype(pt), P0>::value) {
+          const int k = (u - group) / ngroups;          // this pair's k-th unit of problem 0
+          if (A.wave_sync && k > 0) {
+            const int with_k = A.prob[0].raster.num_units - k * ngroups;   // pairs that have a k-th unit
+            wave_barrier(A.wave_sync + (k - 1),
+                         (unsigned int)((PAIR ? 2 : 1) * (with_k < ngroups ? with_k : ngroups)));
+          }
+        }
         return produce_unit<G, PAIR, decltype(pt)>(L, st, rank, pa, tA, tB, u);
       });
   } else if (warp == 1) {

@@ -37,7 +37,7 @@ struct Layout {
   int64_t n_prep_blocks = 0, n_merge_blocks = 0;
   size_t off_status = 0, off_scal = 0, off_mask_part = 0, off_term_part = 0;
   size_t off_tidx = 0, off_tp = 0, off_ent = 0, off_pm = 0, off_ps = 0, off_pg = 0, off_dz = 0;
-  size_t off_rowmap = 0, off_nrows = 0, off_hc = 0, off_dhc = 0;
+  size_t off_rowmap = 0, off_nrows = 0, off_hc = 0, off_dhc = 0, off_wave = 0;
   size_t total = 0;
 };
 
@@ -62,6 +62,7 @@ Layout make_layout(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   L.off_pm = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_wave = take(sizeof(unsigned int) * (size_t)ceil_div(N > 0 ? N : 1, 256) * kMaxSplits);
   L.off_dz = take(2 * (size_t)L.C * L.ldz);   // one dZ chunk (bf16)
   // skipping rows with zero dZ: the kept tokens in order, their count, and
   // one chunk of their H rows and of their dH rows (bf16)
@@ -185,11 +186,13 @@ cudaError_t launch_gemm(int slot, int dev, int groups, const CUtensorMap& ta0, c
 template <class P0>
 cudaError_t launch_one(int slot, int dev, int groups, const CUtensorMap& ta, const CUtensorMap& tb,
                        const CUtensorMap& to, const ProbArgs& pa, Status* status,
-                       const typename P0::Epi::Params& ep, cudaStream_t s, DynRows dyn = DynRows{}) {
+                       const typename P0::Epi::Params& ep, cudaStream_t s, DynRows dyn = DynRows{},
+                       unsigned int* wave_sync = nullptr) {
   GemmArgs a{};
   a.prob[0] = pa;
   a.status = status;
   a.dyn = dyn;
+  a.wave_sync = wave_sync;
   EpiNone::Params none{};
   return launch_gemm<P0, NoProb, kPair>(slot, dev, groups, ta, tb, to, ta, tb, to, a, ep, none, s);
 }
@@ -404,8 +407,13 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const V
   ep.part_m = at<float>(workspace, L.off_pm);
   ep.part_s = at<float>(workspace, L.off_ps);
   ep.part_g = at<float>(workspace, L.off_pg);
+  // wave pacing counters (m_tiles x kMaxSplits >= the number of waves)
+  unsigned int* wave_sync = at<unsigned int>(workspace, L.off_wave);
+  if (cudaMemsetAsync(wave_sync, 0, sizeof(unsigned int) * (size_t)a.raster.m_tiles * kMaxSplits, s) != cudaSuccess)
+    return KD_ERR_CUDA;
   if (!evs.mark()) return KD_ERR_CUDA;
-  if (launch_one<ProbFwd>(0, dev, grid_for(a.raster, groups), tmH, tmW, tmH, a, status, ep, s) != cudaSuccess)
+  if (launch_one<ProbFwd>(0, dev, grid_for(a.raster, groups), tmH, tmW, tmH, a, status, ep, s, DynRows{},
+                          wave_sync) != cudaSuccess)
     return KD_ERR_CUDA;
 
   if (!evs.mark()) return KD_ERR_CUDA;
