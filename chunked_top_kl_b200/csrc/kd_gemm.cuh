@@ -1,17 +1,19 @@
 // Persistent, warp-specialised tcgen05 GEMM with pluggable epilogues.
 //
-// One CTA per SM.  Warp 0 issues TMA loads into a STAGES-deep shared-memory
-// ring, warp 1 issues tcgen05.mma (bf16 x bf16 -> fp32 in tensor memory),
-// warps 2-5 run the epilogue straight out of tensor memory.  Two 128 x 256
-// fp32 accumulators (all 512 TMEM columns) let the epilogue of one tile
-// overlap the MMAs of the next.
+// One CTA per SM, CTA pairs (clusters of two) computing 256 x 256 tiles with
+// cta_group::2 MMAs.  Warp 0 issues TMA loads into a STAGES-deep shared-memory
+// ring, warp 1 of the pair leader issues tcgen05.mma (bf16 x bf16 -> fp32 in
+// tensor memory), warps 2-5 run the epilogue straight out of tensor memory.
+// Two 128 x 256 fp32 accumulators per CTA (all 512 TMEM columns) let the
+// epilogue of one tile overlap the MMAs of the next.
 //
-// Work is a list of units; a unit is one 128-row tile band (m) and a
-// contiguous range of 256-column tiles [n0, n1).  All three roles walk the
-// same unit sequence (u = blockIdx.x, blockIdx.x + gridDim.x, ...), so no
-// scheduling state is shared between them.  The epilogue object lives for a
-// unit, which is what lets the forward epilogue carry a running
-// max / sum-exp across the vocabulary tiles of its range.
+// Work is a list of units; a unit is one tile band (m) and a contiguous range
+// of 256-column tiles [n0, n1).  All three roles walk the same unit sequence
+// (problem 0 round-robin over the pairs, then the pair's share of problem 1;
+// see GemmArgs), so no scheduling state is shared between them.  The
+// epilogue object lives for a unit, which is what lets the forward epilogue
+// carry a running max / sum-exp, and the dZ epilogue its token's scale and
+// teacher cursor, across the tiles of a range.
 #pragma once
 
 #include <cstdint>
@@ -87,11 +89,13 @@ struct GemmArgs {
   JointPlan joint;
   DynRows dyn;
   Status* status;
-  // Optional wave pacing of problem 0 (zeroed counters, one per wave): a
-  // CTA's producer starts its k-th unit only once every CTA with a k-th unit
-  // has issued all loads of its (k-1)-th, so the CTAs that share operand
-  // tiles in a wave keep reading them together.  Pacing only: a wait gives
-  // up after kWaveWaitNs and the CTA goes on.
+  // Optional wave pacing (zeroed counters, one per wave): a CTA's producer
+  // starts its k-th unit of a round-robin only once every CTA with a k-th
+  // unit has issued all loads of its (k-1)-th, so the CTAs that share operand
+  // tiles in a wave keep reading them together.  Counters: problem 0's waves,
+  // then the waves of problem 1's early round-robin (joint.wb of them), then
+  // those of its round-robin over all groups.  Pacing only: a wait gives up
+  // after kWaveWaitNs and the CTA goes on.
   unsigned int* wave_sync;
 };
 
@@ -465,12 +469,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   // This group's units: problem 0 round-robin, then its share of problem 1.
   auto for_each_unit = [&](auto&& body) {
     bool ok = true;
-    for (int u = group; ok && u < A.prob[0].raster.num_units; u += ngroups)
-      ok = body(P0{}, A.prob[0], &tmA0, &tmB0, u);
+    int k = 0;
+    for (int u = group; ok && u < A.prob[0].raster.num_units; u += ngroups, ++k)
+      ok = body(P0{}, A.prob[0], &tmA0, &tmB0, u, k);
     if constexpr (P1::present) {
       const int n1 = joint_count(A.joint, A.prob[1].raster.num_units, ngroups, group);
       for (int i = 0; ok && i < n1; ++i)
-        ok = body(P1{}, A.prob[1], &tmA1, &tmB1, joint_unit(A.joint, ngroups, group, i));
+        ok = body(P1{}, A.prob[1], &tmA1, &tmB1, joint_unit(A.joint, ngroups, group, i), i);
     }
     return ok;
   };
@@ -480,13 +485,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   if (warp == 0) {
     if (lane == 0)
       failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap* tA,
-                                  const CUtensorMap* tB, int u) {
-        if constexpr (std::is_same<decltype(pt), P0>::value) {
-          const int k = (u - group) / ngroups;          // this pair's k-th unit of problem 0
-          if (A.wave_sync && k > 0) {
-            const int with_k = A.prob[0].raster.num_units - k * ngroups;   // pairs that have a k-th unit
-            wave_barrier(A.wave_sync + (k - 1),
-                         (unsigned int)((PAIR ? 2 : 1) * (with_k < ngroups ? with_k : ngroups)));
+                                  const CUtensorMap* tB, int u, int ord) {
+        if (A.wave_sync) {
+          const int cta = PAIR ? 2 : 1;
+          if constexpr (std::is_same<decltype(pt), P0>::value) {
+            // problem 0 round-robin: wave = the pair's unit ordinal
+            if (ord > 0) {
+              const int with_k = A.prob[0].raster.num_units - ord * ngroups;
+              wave_barrier(A.wave_sync + (ord - 1), (unsigned int)(cta * (with_k < ngroups ? with_k : ngroups)));
+            }
+          } else {
+            // problem 1 (joint plan): the early groups' round-robin, then all groups' round-robin
+            const JointPlan& jp = A.joint;
+            const int U1 = A.prob[1].raster.num_units;
+            const int n0w = (A.prob[0].raster.num_units + ngroups - 1) / ngroups;
+            unsigned int* base1 = A.wave_sync + n0w;
+            unsigned int* base2 = base1 + jp.wb;
+            if (group >= jp.r && ord < jp.wb) {
+              if (ord > 0) wave_barrier(base1 + (ord - 1), (unsigned int)(cta * (ngroups - jp.r)));
+            } else {
+              const int j = ord - (group >= jp.r ? jp.wb : 0);
+              if (j > 0) {
+                int with_j = U1 - jp.p2 - j * ngroups;
+                with_j = with_j < 0 ? 0 : (with_j > ngroups ? ngroups : with_j);
+                wave_barrier(base2 + (j - 1), (unsigned int)(cta * with_j));
+              }
+            }
           }
         }
         return produce_unit<G, PAIR, decltype(pt)>(L, st, rank, pa, tA, tB, u);
@@ -494,7 +518,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   } else if (warp == 1) {
     if (lane == 0 && rank == 0)
       failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap*, const CUtensorMap*,
-                                  int u) { return mma_unit<G, PAIR, decltype(pt)>(L, st, tmem_base, pa, u); });
+                                  int u, int) { return mma_unit<G, PAIR, decltype(pt)>(L, st, tmem_base, pa, u); });
   } else {
     const int q = warp & 3;
     const int row = (int)rank * BM + q * 32 + lane;
@@ -504,7 +528,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     EpiCtx cx = make_epi_ctx(L.staging);
     cx.rows_valid = live_rows;
     failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap*, const CUtensorMap*,
-                                int u) {
+                                int u, int) {
       using P = decltype(pt);
       constexpr bool first = std::is_same<P, P0>::value;
       return epi_unit<G, PAIR>(L, st, rank, lane_addr, row, pick<first>(epi0, epi1), pick<first>(ep0, ep1),

@@ -1,9 +1,14 @@
 // Host side of libkdtopkl.so: argument checks, workspace layout, TMA tensor
 // maps, schedules and kernel launches for the fused chunked top-K KL loss.
 //
-// Forward (one call):  teacher_prep -> gemm<EpiFwd> -> lse_merge -> finalize
-// Backward (one call): teacher_prep -> finalize(scale) -> for each chunk of
-//                      tokens: gemm<EpiDz> -> gemm<EpiDh> -> gemm<EpiDw>
+// Forward (one call):  teacher_prep -> gemm<EpiFwd> (wave-paced) -> lse_merge
+//                      -> finalize
+// Backward (one call): teacher_prep -> finalize(scale) [-> compact_rows] ->
+//                      for each chunk of tokens: [gather_rows ->]
+//                      gemm<EpiDz> -> gemm<EpiDh + EpiDw> [-> scatter_rows]
+//                      (bracketed steps: skipping masked rows)
+// Teacher top-K cache writer: for each chunk, gemm<EpiDw, fp32 store> ->
+//                      topk_select
 // The fused chunked loss of "Efficient Knowledge Distillation for LLMs"
 // (Japanese summary, method paragraph) projects, normalises and gathers one
 // chunk at a time and recomputes each chunk in the backward pass; here the
@@ -37,7 +42,8 @@ struct Layout {
   int64_t n_prep_blocks = 0, n_merge_blocks = 0;
   size_t off_status = 0, off_scal = 0, off_mask_part = 0, off_term_part = 0;
   size_t off_tidx = 0, off_tp = 0, off_ent = 0, off_pm = 0, off_ps = 0, off_pg = 0, off_dz = 0;
-  size_t off_rowmap = 0, off_nrows = 0, off_hc = 0, off_dhc = 0, off_wave = 0;
+  size_t off_rowmap = 0, off_nrows = 0, off_hc = 0, off_dhc = 0, off_wave = 0, off_jwave = 0;
+  int64_t jwave_per_chunk = 0;
   size_t total = 0;
 };
 
@@ -63,6 +69,9 @@ Layout make_layout(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_wave = take(sizeof(unsigned int) * (size_t)ceil_div(N > 0 ? N : 1, 256) * kMaxSplits);
+  // joint launches' wave counters: per chunk, up to 2 (U0 + U1) + 4
+  L.jwave_per_chunk = 2 * (ceil_div(L.C, 256) * ceil_div(d, 256) + ceil_div(V, 256) * ceil_div(d, 256)) + 4;
+  L.off_jwave = take(sizeof(unsigned int) * (size_t)L.jwave_per_chunk * ceil_div(N > 0 ? N : 1, L.C));
   L.off_dz = take(2 * (size_t)L.C * L.ldz);   // one dZ chunk (bf16)
   // skipping rows with zero dZ: the kept tokens in order, their count, and
   // one chunk of their H rows and of their dH rows (bf16)
@@ -500,6 +509,10 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     return KD_ERR_CUDA;
   const int groups = resident_groups(dev);
   const unsigned copy_blocks = (unsigned)(device_sms(dev) * 8);
+  unsigned int* jwave = at<unsigned int>(workspace, L.off_jwave);
+  if (cudaMemsetAsync(jwave, 0, sizeof(unsigned int) * (size_t)L.jwave_per_chunk * ceil_div(N, chunk), s) !=
+      cudaSuccess)
+    return KD_ERR_CUDA;
 
   for (int64_t c0 = 0; c0 < N; c0 += chunk) {
     const int64_t Cc = (N - c0 < chunk) ? (N - c0) : chunk;
@@ -560,6 +573,7 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     a45.prob[1].b_k0 = hrow0;
     a45.prob[1].dyn_role = 2;
     plan_second_problem(a45, groups);
+    a45.wave_sync = jwave + (size_t)(c0 / chunk) * L.jwave_per_chunk;
     EpiDh::Params e4{};
     e4.row0 = hrow0;
     EpiDw::Params e5{};
