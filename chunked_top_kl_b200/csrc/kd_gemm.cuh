@@ -89,13 +89,11 @@ struct GemmArgs {
   JointPlan joint;
   DynRows dyn;
   Status* status;
-  // Optional wave pacing (zeroed counters, one per wave): a CTA's producer
-  // starts its k-th unit of a round-robin only once every CTA with a k-th
-  // unit has issued all loads of its (k-1)-th, so the CTAs that share operand
-  // tiles in a wave keep reading them together.  Counters: problem 0's waves,
-  // then the waves of problem 1's early round-robin (joint.wb of them), then
-  // those of its round-robin over all groups.  Pacing only: a wait gives up
-  // after kWaveWaitNs and the CTA goes on.
+  // Optional wave pacing (zeroed counters, wave_slots_bound of them; see
+  // wave_slot): a CTA's producer starts a wave of a round-robin only once
+  // every CTA with that wave has issued all loads of the previous one, so the
+  // CTAs that share operand tiles keep reading them together.  Pacing only: a
+  // wait gives up after kWaveWaitNs and the CTA goes on.
   unsigned int* wave_sync;
 };
 
@@ -487,31 +485,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       failed = !for_each_unit([&](auto pt, const ProbArgs& pa, const CUtensorMap* tA,
                                   const CUtensorMap* tB, int u, int ord) {
         if (A.wave_sync) {
-          const int cta = PAIR ? 2 : 1;
-          if constexpr (std::is_same<decltype(pt), P0>::value) {
-            // problem 0 round-robin: wave = the pair's unit ordinal
-            if (ord > 0) {
-              const int with_k = A.prob[0].raster.num_units - ord * ngroups;
-              wave_barrier(A.wave_sync + (ord - 1), (unsigned int)(cta * (with_k < ngroups ? with_k : ngroups)));
-            }
-          } else {
-            // problem 1 (joint plan): the early groups' round-robin, then all groups' round-robin
-            const JointPlan& jp = A.joint;
-            const int U1 = A.prob[1].raster.num_units;
-            const int n0w = (A.prob[0].raster.num_units + ngroups - 1) / ngroups;
-            unsigned int* base1 = A.wave_sync + n0w;
-            unsigned int* base2 = base1 + jp.wb;
-            if (group >= jp.r && ord < jp.wb) {
-              if (ord > 0) wave_barrier(base1 + (ord - 1), (unsigned int)(cta * (ngroups - jp.r)));
-            } else {
-              const int j = ord - (group >= jp.r ? jp.wb : 0);
-              if (j > 0) {
-                int with_j = U1 - jp.p2 - j * ngroups;
-                with_j = with_j < 0 ? 0 : (with_j > ngroups ? ngroups : with_j);
-                wave_barrier(base2 + (j - 1), (unsigned int)(cta * with_j));
-              }
-            }
-          }
+          constexpr int prob = std::is_same<decltype(pt), P0>::value ? 0 : 1;
+          int expected = 0;
+          const int slot = wave_slot(prob, ord, group, ngroups, A.prob[0].raster.num_units,
+                                     P1::present ? A.prob[1].raster.num_units : 0, A.joint, &expected);
+          if (slot >= 0) wave_barrier(A.wave_sync + slot, (unsigned int)((PAIR ? 2 : 1) * expected));
         }
         return produce_unit<G, PAIR, decltype(pt)>(L, st, rank, pa, tA, tB, u);
       });

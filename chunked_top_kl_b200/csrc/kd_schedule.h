@@ -143,4 +143,41 @@ KD_HD int joint_unit(const JointPlan& p, int groups, int g, int i) {
   return p.p2 + gp + i * groups;
 }
 
+// Wave pacing.  In a round-robin over `groups`, the groups that hold their
+// j-th unit at the same time share operand tiles; a counter per wave lets
+// every group start its j-th unit only once all groups with a j-th unit have
+// finished issuing their (j-1)-th.  Counters: problem 0's waves, then those
+// of problem 1's early round-robin (joint plan, groups >= r), then those of
+// its round-robin over all groups.  Launches whose units are shorter than
+// kPaceKBlocks K blocks are not paced (the waits then cost more than the
+// shared reads save).
+constexpr int kPaceKBlocks = 64;
+
+// Counter index that group `group` waits on before its ord-th unit of
+// problem `prob` (0 or 1), and the number of groups that arrive there
+// (*expected); -1 when that unit starts its round-robin.  U1 = 0 and jp = {}
+// for a launch of problem 0 alone.
+KD_HD int wave_slot(int prob, int ord, int group, int groups, int U0, int U1, const JointPlan& jp,
+                    int* expected) {
+  auto clampg = [&](int64_t v) { return (int)(v < 0 ? 0 : (v > groups ? groups : v)); };
+  const int w0 = (int)ceil_div64(U0, groups);                         // problem 0's waves
+  if (prob == 0) {
+    if (ord == 0) return -1;
+    *expected = clampg((int64_t)U0 - (int64_t)ord * groups);
+    return ord - 1;
+  }
+  if (group >= jp.r && ord < jp.wb) {
+    if (ord == 0) return -1;
+    *expected = groups - jp.r;
+    return w0 + ord - 1;
+  }
+  const int j = ord - (group >= jp.r ? jp.wb : 0);
+  if (j == 0) return -1;
+  *expected = clampg((int64_t)U1 - jp.p2 - (int64_t)j * groups);
+  return w0 + jp.wb + j - 1;
+}
+
+// Counters a launch needs: an upper bound of every index wave_slot returns, plus one.
+KD_HD int64_t wave_slots_bound(int64_t U0, int64_t U1) { return 2 * (U0 + U1) + 4; }
+
 }  // namespace kd

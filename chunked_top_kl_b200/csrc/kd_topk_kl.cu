@@ -68,9 +68,9 @@ Layout make_layout(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   L.off_pm = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
   L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
-  L.off_wave = take(sizeof(unsigned int) * (size_t)ceil_div(N > 0 ? N : 1, 256) * kMaxSplits);
-  // joint launches' wave counters: per chunk, up to 2 (U0 + U1) + 4
-  L.jwave_per_chunk = 2 * (ceil_div(L.C, 256) * ceil_div(d, 256) + ceil_div(V, 256) * ceil_div(d, 256)) + 4;
+  // wave counters: the forward's, and per chunk the joint launch's
+  L.off_wave = take(sizeof(unsigned int) * (size_t)wave_slots_bound(ceil_div(N > 0 ? N : 1, 256) * kMaxSplits, 0));
+  L.jwave_per_chunk = wave_slots_bound(ceil_div(L.C, 256) * ceil_div(d, 256), ceil_div(V, 256) * ceil_div(d, 256));
   L.off_jwave = take(sizeof(unsigned int) * (size_t)L.jwave_per_chunk * ceil_div(N > 0 ? N : 1, L.C));
   L.off_dz = take(2 * (size_t)L.C * L.ldz);   // one dZ chunk (bf16)
   // skipping rows with zero dZ: the kept tokens in order, their count, and
@@ -416,9 +416,10 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const V
   ep.part_m = at<float>(workspace, L.off_pm);
   ep.part_s = at<float>(workspace, L.off_ps);
   ep.part_g = at<float>(workspace, L.off_pg);
-  // wave pacing counters (m_tiles x kMaxSplits >= the number of waves)
+  // wave pacing counters
   unsigned int* wave_sync = at<unsigned int>(workspace, L.off_wave);
-  if (cudaMemsetAsync(wave_sync, 0, sizeof(unsigned int) * (size_t)a.raster.m_tiles * kMaxSplits, s) != cudaSuccess)
+  if (cudaMemsetAsync(wave_sync, 0, sizeof(unsigned int) * (size_t)wave_slots_bound(a.raster.num_units, 0), s) !=
+      cudaSuccess)
     return KD_ERR_CUDA;
   if (!evs.mark()) return KD_ERR_CUDA;
   if (launch_one<ProbFwd>(0, dev, grid_for(a.raster, groups), tmH, tmW, tmH, a, status, ep, s, DynRows{},
@@ -573,7 +574,8 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     a45.prob[1].b_k0 = hrow0;
     a45.prob[1].dyn_role = 2;
     plan_second_problem(a45, groups);
-    a45.wave_sync = jwave + (size_t)(c0 / chunk) * L.jwave_per_chunk;
+    if (a45.prob[1].num_kb >= kPaceKBlocks)     // dW tiles long enough to pace (see wave_slot)
+      a45.wave_sync = jwave + (size_t)(c0 / chunk) * L.jwave_per_chunk;
     EpiDh::Params e4{};
     e4.row0 = hrow0;
     EpiDw::Params e5{};

@@ -89,6 +89,40 @@ int main() {
             }
             ++cases;
           }
+  // wave pacing: every counter a group waits on receives exactly the number
+  // of arrivals it waits for (else the barrier would time out), all waits
+  // on one counter expect the same number, and indices stay in bounds
+  const long ks0[] = {1, 45, 3142};
+  for (long U0 : U0s)
+    for (long k0 : ks0)
+      for (long U1 : U1s)
+        for (long k1 : k1s)
+          for (int g : {1, 7, 74, 148}) {
+            const JointPlan p = joint_plan(U0, k0, U1, k1, g);
+            const long cap = wave_slots_bound(U0, U1);
+            std::vector<int> arrivals((size_t)cap, 0), want((size_t)cap, -1);
+            for (int grp = 0; grp < g; ++grp) {
+              const long n0 = grp < U0 ? (U0 - grp + g - 1) / g : 0;
+              const int n1 = joint_count(p, U1, g, grp);
+              for (int prob = 0; prob < 2; ++prob)
+                for (long ord = 0; ord < (prob == 0 ? n0 : n1); ++ord) {
+                  int e = 0;
+                  const int slot = wave_slot(prob, (int)ord, grp, g, (int)U0, (int)U1, p, &e);
+                  if (slot < 0) continue;
+                  if (slot >= cap) { printf("FAIL pace slot %d >= %ld\n", slot, cap); return 1; }
+                  if (want[(size_t)slot] >= 0 && want[(size_t)slot] != e) { printf("FAIL pace expected\n"); return 1; }
+                  want[(size_t)slot] = e;
+                  ++arrivals[(size_t)slot];
+                }
+            }
+            for (long i = 0; i < cap; ++i)
+              if (want[(size_t)i] >= 0 && arrivals[(size_t)i] != want[(size_t)i]) {
+                printf("FAIL pace U0 %ld k0 %ld U1 %ld k1 %ld g %d: slot %ld %d arrivals for %d\n", U0, k0, U1, k1,
+                       g, i, arrivals[(size_t)i], want[(size_t)i]);
+                return 1;
+              }
+            ++cases;
+          }
   printf("OK %d\n", cases);
   return 0;
 }
