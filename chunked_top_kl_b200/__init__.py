@@ -11,7 +11,7 @@ from ._abi import (EXPORTS, KDError, kd_status_string, kd_teacher_topk, kd_teach
                    kd_topk_kl_backward, kd_topk_kl_backward_ex, kd_topk_kl_backward_profiled, kd_topk_kl_check,
                    kd_topk_kl_forward, kd_topk_kl_forward_backward, kd_topk_kl_forward_backward_ex,
                    kd_topk_kl_forward_ex, kd_topk_kl_forward_noalloc, kd_topk_kl_workspace_size, load,
-                   make_options)
+                   kd_selftest_wait_timeout, make_options)
 from .api import (KDTopKKLFunction, alloc_workspace, backward, backward_launches, check, forward,
                   forward_backward, forward_backward_launches, kd_topk_kl_loss, teacher_topk, workspace_bytes)
 
@@ -19,7 +19,7 @@ __all__ = [
     "EXPORTS", "KDError", "kd_status_string", "kd_teacher_topk", "kd_teacher_topk_workspace_size",
     "kd_topk_kl_backward", "kd_topk_kl_backward_ex", "kd_topk_kl_backward_profiled", "kd_topk_kl_check",
     "kd_topk_kl_forward", "kd_topk_kl_forward_backward", "kd_topk_kl_forward_backward_ex", "kd_topk_kl_forward_ex",
-    "kd_topk_kl_forward_noalloc", "kd_topk_kl_workspace_size", "load", "make_options",
+    "kd_topk_kl_forward_noalloc", "kd_topk_kl_workspace_size", "kd_selftest_wait_timeout", "load", "make_options",
     "KDTopKKLFunction", "alloc_workspace", "backward", "backward_launches", "check", "forward",
     "forward_backward", "forward_backward_launches", "kd_topk_kl_loss", "teacher_topk", "workspace_bytes",
 ]

@@ -34,6 +34,7 @@ EXPORTS = (
     "kd_topk_kl_forward_backward_ex",
     "kd_teacher_topk_workspace_size",
     "kd_teacher_topk",
+    "kd_selftest_wait_timeout",
 )
 
 
@@ -97,6 +98,8 @@ def load() -> ctypes.CDLL:
         lib.kd_teacher_topk_workspace_size.restype = sz
         lib.kd_teacher_topk.argtypes = [p, p, i64, i64, i64, i64, i64, p, p, p, sz, p]
         lib.kd_teacher_topk.restype = i32
+        lib.kd_selftest_wait_timeout.argtypes = [p, sz, i64, p]
+        lib.kd_selftest_wait_timeout.restype = i32
         _lib = lib
     return _lib
 
@@ -210,3 +213,8 @@ def kd_teacher_topk_workspace_size(N: int, d: int, V: int, K: int, chunk: int) -
 def kd_teacher_topk(Ht, Wt, N, d, V, K, chunk, topk_idx, topk_logit, workspace, workspace_bytes, stream) -> int:
     return int(load().kd_teacher_topk(Ht, Wt, N, d, V, K, chunk, topk_idx, topk_logit, workspace,
                                       workspace_bytes, stream))
+
+
+def kd_selftest_wait_timeout(workspace, workspace_bytes, limit_us, stream) -> int:
+    """Launch the failure-detection self-test (see the C header)."""
+    return int(load().kd_selftest_wait_timeout(workspace, workspace_bytes, int(limit_us), stream))

@@ -782,6 +782,40 @@ int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- failure-detection self-test
+//
+// Every pipeline wait in the kernels is bounded: when a barrier phase does not
+// complete in time, the waiting thread gives up, the kernel records a timeout
+// in the workspace's status words, lets issued copies land and exits, and
+// kd_topk_kl_check reports KD_ERR_TIMEOUT.  This kernel exercises that path
+// on purpose: it waits on an mbarrier that nothing ever arrives on.
+
+namespace {
+
+__global__ void wait_selftest_kernel(Status* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_barrier_init();
+    abort_flag = 0;
+    if (!mbar_wait_bounded(b, 0, &abort_flag, limit_ns)) atomicOr(&status->timeout, 1u);
+  }
+}
+
+}  // namespace
+
+extern "C" int kd_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_us, void* stream) {
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < sizeof(Status)) return KD_ERR_INVALID_ARG;
+  if (limit_us < 1 || limit_us > 2000000) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Status* status = at<Status>(workspace, 0);
+  if (cudaMemsetAsync(status, 0, sizeof(Status), s) != cudaSuccess) return KD_ERR_CUDA;
+  wait_selftest_kernel<<<1, 32, 0, s>>>(status, (uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? KD_OK : KD_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- forward without a workspace
 //
 // Some callers cannot allocate device memory at the point where they need

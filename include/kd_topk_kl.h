@@ -260,6 +260,17 @@ int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_
                     int64_t chunk, int32_t* topk_idx, float* topk_logit,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Failure-detection self-test.  Every pipeline wait in the kernels is
+ * bounded: a barrier phase that does not complete within its limit makes the
+ * waiting kernel record a timeout in the workspace's status words and exit,
+ * and kd_topk_kl_check then returns KD_ERR_TIMEOUT; the device stays usable.
+ * This call exercises that path: it clears the status words and launches a
+ * kernel that waits on a barrier nothing ever arrives on, with a limit of
+ * limit_us microseconds (1 .. 2,000,000).  Any workspace of this library
+ * (>= 256 bytes, 256-byte aligned) will do; the next call on it clears the
+ * status again. */
+int kd_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_us, void* stream);
+
 /* Synchronises `stream`, then reads the device-side status words that the
  * last forward or backward call on this workspace wrote.  Returns KD_OK,
  * KD_ERR_BAD_INDEX (teacher index outside [0, V) seen), KD_ERR_TIMEOUT (a
