@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB_DIR = os.path.join(HERE, "_lib")
 LIB = os.path.join(LIB_DIR, "libkdtopkl.so")
 SOURCES = ["kd_topk_kl.cu"]
-HEADERS = ["kd_ptx.cuh", "kd_gemm.cuh", "kd_small_kernels.cuh", "kd_schedule.h"]
+HEADERS = ["kd_ptx.cuh", "kd_gemm.cuh", "kd_small_kernels.cuh", "kd_schedule.h", "kd_topk_select.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

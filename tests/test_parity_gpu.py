@@ -91,6 +91,8 @@ SMALL_CASES = [
     (1, 64, 24, 5, 2.0, 4096, "ones"),                # single token, V < one tile
     (700, 512, 5000, 100, 1.3, 256, "drop5"),         # K = 100, many tiles
     (256, 8, 300, 300, 1.0, 128, "ones"),             # K = V (whole vocabulary), d = 8
+    (300, 320, 2000, 12, 1.1, 128, "drop5"),          # d = 256 + 64: a narrow last column tile of dH / dW
+    (260, 384, 1500, 9, 1.0, 128, "ones"),            # d = 256 + 128: a last column tile exactly half wide
 ]
 
 
