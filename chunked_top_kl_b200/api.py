@@ -15,9 +15,39 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _check_buffer(t, name: str, shape, dtype, dev) -> None:
+    """A caller-supplied tensor the library reads or writes through a raw
+    pointer: it must be on ``dev`` with exactly this shape and dtype, and
+    contiguous, or the kernels would address memory outside it."""
+    if t.device != dev:
+        raise ValueError(f"kd_topk_kl: {name} is on {t.device}, the inputs on {dev}")
+    if t.dtype != dtype:
+        raise TypeError(f"kd_topk_kl: {name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"kd_topk_kl: {name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"kd_topk_kl: {name} must be contiguous")
+
+
+def _check_workspace(ws, dev) -> None:
+    if ws.device != dev or ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous():
+        raise ValueError(f"kd_topk_kl: workspace must be a contiguous 1-D uint8 tensor on {dev}")
+
+
+def _grad_scalar(grad_loss, dev):
+    if grad_loss is None:
+        return None
+    if grad_loss.numel() != 1:
+        raise ValueError("kd_topk_kl: grad_loss must hold one value")
+    return grad_loss.reshape(()).to(device=dev, dtype=torch.float32).contiguous()
+
+
 def _check_inputs(H, W, topk_idx, topk_logit, mask):
     if not (H.is_cuda and W.is_cuda and topk_idx.is_cuda and topk_logit.is_cuda):
         raise ValueError("kd_topk_kl: all inputs must be CUDA tensors")
+    for t in (W, topk_idx, topk_logit) + ((mask,) if mask is not None else ()):
+        if t.device != H.device:
+            raise ValueError(f"kd_topk_kl: inputs on {t.device} and {H.device}; all must be on one device")
     if H.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
         raise TypeError("kd_topk_kl: H and W must be bfloat16")
     if topk_idx.dtype != torch.int32 or topk_logit.dtype not in (torch.float32, torch.bfloat16):
@@ -85,6 +115,7 @@ def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 
     dev = H.device
     if workspace is None:
         workspace = alloc_workspace(N, d, V, K, chunk, dev)
+    _check_workspace(workspace, dev)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     lse = torch.empty(N, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
@@ -123,13 +154,16 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
     dev = H.device
     if workspace is None:
         workspace = alloc_workspace(N, d, V, K, chunk, dev)
+    _check_workspace(workspace, dev)
+    _check_buffer(lse, "lse", (N,), torch.float32, dev)
     if dH is None:
         dH = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    _check_buffer(dH, "dH", (N, d), torch.bfloat16, dev)
     if dW is None:
         dW = torch.empty((V, d), dtype=torch.float32, device=dev)
         accumulate_dW = False
-    if grad_loss is not None:
-        grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
+    _check_buffer(dW, "dW", (V, d), torch.float32, dev)
+    grad_loss = _grad_scalar(grad_loss, dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     opt = _options(topk_logit, student_temperature, skip_masked_rows)
     if opt is not None:
@@ -170,15 +204,17 @@ def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chun
     dev = H.device
     if workspace is None:
         workspace = alloc_workspace(N, d, V, K, chunk, dev)
+    _check_workspace(workspace, dev)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     lse = torch.empty(N, dtype=torch.float32, device=dev)
     if dH is None:
         dH = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    _check_buffer(dH, "dH", (N, d), torch.bfloat16, dev)
     if dW is None:
         dW = torch.empty((V, d), dtype=torch.float32, device=dev)
         accumulate_dW = False
-    if grad_loss is not None:
-        grad_loss = grad_loss.to(device=dev, dtype=torch.float32).contiguous()
+    _check_buffer(dW, "dW", (V, d), torch.float32, dev)
+    grad_loss = _grad_scalar(grad_loss, dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     evs = _event_handles(events)
     opt = _options(topk_logit, student_temperature, skip_masked_rows)
@@ -201,6 +237,8 @@ def teacher_topk(Ht, Wt, K: int, chunk: int = 1024,
         raise TypeError("teacher_topk: Ht and Wt must be bfloat16 CUDA tensors")
     if not (Ht.is_contiguous() and Wt.is_contiguous()) or Ht.shape[1] != Wt.shape[1]:
         raise ValueError("teacher_topk: contiguous Ht [N,d] and Wt [V,d] expected")
+    if Wt.device != Ht.device:
+        raise ValueError("teacher_topk: Ht and Wt must be on one device")
     N, d = Ht.shape
     V = Wt.shape[0]
     dev = Ht.device
@@ -209,6 +247,7 @@ def teacher_topk(Ht, Wt, K: int, chunk: int = 1024,
         if n == 0:
             raise ValueError("teacher_topk: unsupported sizes")
         workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    _check_workspace(workspace, dev)
     idx = torch.empty((N, K), dtype=torch.int32, device=dev)
     val = torch.empty((N, K), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream

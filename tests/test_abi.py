@@ -113,3 +113,32 @@ def test_options_are_validated_first(lib):
                                                P, nb, None, None, bad) == _abi.KD_ERR_INVALID_ARG
     # fp32 logits need 4-byte alignment (rejected before anything is enqueued)
     assert fwd(_abi.make_options(), logit=P + 2) == _abi.KD_ERR_INVALID_ARG
+
+
+def test_binding_checks_caller_buffers(lib):
+    """Buffers the caller hands in (dH, dW, lse, workspace, grad_loss) are
+    written or read through raw pointers, so the binding checks device, shape,
+    dtype and contiguity before any call (host logic, CPU tensors here)."""
+    import torch
+    from chunked_top_kl_b200 import api
+    cpu = torch.device("cpu")
+    api._check_buffer(torch.empty(4, 8, dtype=torch.bfloat16), "dH", (4, 8), torch.bfloat16, cpu)
+    with pytest.raises(ValueError, match="shape"):
+        api._check_buffer(torch.empty(4, 9, dtype=torch.bfloat16), "dH", (4, 8), torch.bfloat16, cpu)
+    with pytest.raises(TypeError):
+        api._check_buffer(torch.empty(4, 8, dtype=torch.float32), "dH", (4, 8), torch.bfloat16, cpu)
+    with pytest.raises(ValueError, match="contiguous"):
+        api._check_buffer(torch.empty(8, 4, dtype=torch.bfloat16).t(), "dH", (4, 8), torch.bfloat16, cpu)
+    with pytest.raises(ValueError, match="is on"):
+        api._check_buffer(torch.empty(4, 8, dtype=torch.bfloat16), "dH", (4, 8), torch.bfloat16,
+                          torch.device("meta"))
+    api._check_workspace(torch.empty(64, dtype=torch.uint8), cpu)
+    for bad in (torch.empty(64, dtype=torch.int8), torch.empty(8, 8, dtype=torch.uint8),
+                torch.empty(128, dtype=torch.uint8)[::2]):
+        with pytest.raises(ValueError):
+            api._check_workspace(bad, cpu)
+    assert api._grad_scalar(None, cpu) is None
+    g = api._grad_scalar(torch.tensor([2.5], dtype=torch.float64), cpu)
+    assert g.shape == () and g.dtype == torch.float32 and float(g) == 2.5
+    with pytest.raises(ValueError):
+        api._grad_scalar(torch.ones(2), cpu)

@@ -270,3 +270,23 @@ def test_event_count_is_checked(kd):
     with pytest.raises(kd.KDError):
         kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws,
                             events=too_few)
+
+
+def test_caller_buffers_are_checked(kd):
+    """A dH, dW or lse of the wrong shape or dtype is refused before any launch."""
+    x = workloads.make_inputs(_cfg(130, 64, 600, 4, seed=15))
+    g = _to_dev(x)
+    ws = kd.alloc_workspace(130, 64, 600, 4, 64, "cuda")
+    _, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws)
+    args = (g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64)
+    with pytest.raises(ValueError):
+        kd.backward(*args, lse, workspace=ws, dH=torch.empty(129, 64, dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(TypeError):
+        kd.backward(*args, lse, workspace=ws, dW=torch.empty(600, 64, dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        kd.backward(*args, lse[:-1], workspace=ws)
+    with pytest.raises(ValueError):
+        kd.forward_backward(*args, workspace=ws, dW=torch.empty(600, 64, device="cpu"))
+    torch.cuda.synchronize()
+    dH, dW = kd.backward(*args, lse, workspace=ws)     # the same call with valid buffers still runs
+    assert kd.check(ws) == (0, 0) and torch.isfinite(dW).all()
