@@ -9,6 +9,7 @@ in HBM before the timed region starts.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--N TOKENS]
   python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host
+  python bench.py --op teacher-topk ...     # the offline teacher top-K cache writer
 
 For N > 1 it runs under torch.distributed.run, one process per GPU; each
 rank computes an independent replica (the path has no exchange step), the
@@ -467,6 +468,114 @@ def run_cuda(args, cfg, world, rank, local):
     return 0
 
 
+TOPK_METRIC = "teacher top-K cache write tokens/s (logits GEMM + exact top-K select)"
+
+
+def topk_launches_per_call(N: int, chunk: int) -> int:
+    """Kernel launches of one kd_teacher_topk call: per chunk, the logits GEMM and the select."""
+    return 0 if N == 0 else 2 * ((N + chunk - 1) // chunk)
+
+
+def run_teacher_topk(args, cfg, world, rank, local):
+    """The offline cache writer: a teacher head [V, d] over N hidden states,
+    top-K (index, logit) per token.  One step = one kd_teacher_topk call over
+    the whole batch; the workload's H and W stand in for the teacher's."""
+    import chunked_top_kl_b200 as kd
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    rcfg = cfg if rank == 0 else cfg.__class__(**{**cfg.__dict__, "seed": cfg.seed + 1000 * rank})
+    x = workloads.make_inputs(rcfg)
+    N, d, V, K, chunk = cfg.N, cfg.d, cfg.V, cfg.K, args.topk_chunk
+    Ht, Wt = x["H"].to(dev), x["W"].to(dev)
+    n_ws = kd.kd_teacher_topk_workspace_size(N, d, V, K, chunk)
+    ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        kd.teacher_topk(Ht, Wt, K, chunk=chunk, workspace=ws)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local) if not args.no_clocks else None
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        idx, val = kd.teacher_topk(Ht, Wt, K, chunk=chunk, workspace=ws)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    ms = reduce_max(start.elapsed_time(end), world, dev)
+
+    e2e = None
+    if not args.no_e2e:
+        hH, hW = x["H"].pin_memory(), x["W"].pin_memory()
+        oi = torch.empty((N, K), dtype=torch.int32).pin_memory()
+        ov = torch.empty((N, K), dtype=torch.float32).pin_memory()
+
+        def e2e_steps(n):
+            for _ in range(n):
+                Ht.copy_(hH, non_blocking=True)
+                Wt.copy_(hW, non_blocking=True)
+                i, v = kd.teacher_topk(Ht, Wt, K, chunk=chunk, workspace=ws)
+                oi.copy_(i, non_blocking=True)
+                ov.copy_(v, non_blocking=True)
+
+        e2e_steps(args.warmup)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        s2 = torch.cuda.Event(enable_timing=True)
+        e2 = torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        e2e_steps(args.steps)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e2e_ms = reduce_max(s2.elapsed_time(e2), world, dev)
+        e2e = {"value": N * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(hH.numel() * 2 + hW.numel() * 2),
+               "d2h_bytes_per_step": int(oi.numel() * 4 + ov.numel() * 4), "ms_per_step": e2e_ms / args.steps}
+    if rank != 0:
+        return 0
+
+    peaks, peaks_src = load_peaks()
+    ms_step = ms / args.steps
+    gemm_tflops = 2.0 * N * d * V / (ms_step / 1e3) / 1e12
+    peak_sus = peaks["bf16_tflops_sustained"]
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n = int(max(1, min(N, args.topk_cpu_rows)))
+        t0 = time.perf_counter()
+        oracle.teacher_topk(x["H"][:n], x["W"], K)
+        t = time.perf_counter() - t0
+        cpu = {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {n} of {N} tokens (full teacher head), fp64 logits + stable sort, {t:.1f} s"}
+    line = {
+        "metric": TOPK_METRIC, "value": N * world * args.steps / (ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 -> f32",
+        "data": "synthetic (seeded; Ht~N(0,1), Wt~N(0,0.02^2) bf16)",
+        "config": {"workload": f"teacher_topk_{cfg.name}", "N": N, "d": d, "V": V, "K": K, "chunk": chunk,
+                   "seed": cfg.seed, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (Wt > 126 MB); no flush"},
+        "clocks": clocks,
+        "gpu_launches": topk_launches_per_call(N, chunk) * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "whole call (logits GEMM + select)",
+                     "achieved": gemm_tflops, "peak": peak_sus, "unit": "TFLOP/s", "frac": gemm_tflops / peak_sus,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks_src})",
+                     "flops_per_call": 2.0 * N * d * V, "traffic": None},
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,9 +592,15 @@ def main(argv=None):
                          "(same results; auto: kept when some token is masked and N >= %d)" % AUTO_SKIP_MIN_N)
     ap.add_argument("--cpu-flops", type=float, default=4e12, help="oracle work for cpu_baseline")
     ap.add_argument("--ref-flops", type=float, default=1.2e12, help="oracle work per reference step")
+    ap.add_argument("--op", choices=["loss", "teacher-topk"], default="loss",
+                    help="loss: the fused loss step (default); teacher-topk: the offline cache writer")
+    ap.add_argument("--topk-chunk", type=int, default=4096, help="tokens per chunk of the cache writer")
+    ap.add_argument("--topk-cpu-rows", type=int, default=256, help="oracle tokens for its cpu_baseline")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.op == "teacher-topk" and args.impl == "reference":
+        ap.error("--op teacher-topk times the library; its oracle is timed in cpu_baseline")
     cfg = workloads.get_config(args.config, args.N)
     world, rank, local = dist_setup(args.impl)
     if world != args.gpus and args.impl == "cuda":
@@ -493,6 +608,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, cfg, world, rank)
+        if args.op == "teacher-topk":
+            return run_teacher_topk(args, cfg, world, rank, local)
         return run_cuda(args, cfg, world, rank, local)
     finally:
         if world > 1 and args.impl == "cuda":

@@ -80,3 +80,14 @@ def test_reference_arm_other_ranks_exit_quietly():
 def test_warmup_below_three_rejected():
     out = _run_bench(["--impl", "reference", "--config", "0", "--steps", "1", "--warmup", "2"])
     assert out.returncode != 0
+
+
+def test_teacher_topk_mode_host_logic():
+    import bench
+    assert bench.topk_launches_per_call(32768, 4096) == 16
+    assert bench.topk_launches_per_call(4097, 4096) == 4
+    assert bench.topk_launches_per_call(0, 4096) == 0
+    # the cache writer has no reference arm of its own (its oracle is the cpu_baseline)
+    out = _run_bench(["--op", "teacher-topk", "--impl", "reference", "--config", "0", "--steps", "1",
+                      "--warmup", "3"])
+    assert out.returncode != 0 and "teacher-topk" in out.stderr
