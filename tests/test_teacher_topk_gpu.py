@@ -89,3 +89,22 @@ def test_workspace_and_arguments(kd):
     assert kd.kd_teacher_topk_workspace_size(1000, 64, 50, 100, 256) == 0       # K > V
     assert kd.kd_teacher_topk_workspace_size(1000, 60, 5000, 100, 256) == 0     # d % 8
     assert kd.kd_teacher_topk_workspace_size(1000, 64, 5000, 513, 256) == 0     # K > 512
+
+
+@pytest.mark.parametrize("V,K,n_pos", [(5000, 10, 0), (3000, 512, 0), (3020, 100, 20)],
+                         ids=["all_tied_K10", "all_tied_K512", "20_above_3000_tied"])
+def test_tied_rows(kd, V, K, n_pos):
+    """Rows where more values share the K-th value's 12-bit key bin than the
+    select's shared-memory candidate buffer holds (2048): it then finishes as a
+    radix select, with the same result (ties in increasing column order)."""
+    g = torch.Generator().manual_seed(V + K)
+    N, d = 37, 16
+    Ht = torch.randint(1, 3, (N, d), generator=g).to(torch.bfloat16)       # positive
+    Wt = torch.zeros(V, d, dtype=torch.bfloat16)
+    if n_pos:
+        # n_pos columns near the end with positive logits; every other logit is 0
+        Wt[V - n_pos:] = torch.randint(1, 3, (n_pos, d), generator=g).to(torch.bfloat16)
+    idx, val = _gpu_topk(kd, Ht, Wt, K, chunk=16)
+    ridx, rval = oracle.teacher_topk(Ht, Wt, K)
+    assert np.array_equal(idx, ridx)
+    assert np.array_equal(val.astype(np.float64), rval)
