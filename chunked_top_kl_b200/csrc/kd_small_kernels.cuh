@@ -170,16 +170,30 @@ teacher_prep_kernel(const int32_t* __restrict__ idx, const void* __restrict__ lo
 //   term = tfac * (sum p log p - zscale * sum p z + P * lse)
 // with P = 1, or 0 for a token without teacher entries (its prepared row
 // starts with kSentinel), and tfac = 1 or T^2.
+//
+// `poison_on` (may be null): status words that earlier kernels of the same
+// pass on this stream have set.  When any of them reports a bad teacher
+// index or a timed-out wait, every lse is written as NaN, for callers that
+// have no way to read the status words themselves.
+__device__ __forceinline__ bool status_failed(const Status* s) {
+  if (!s) return false;
+  const volatile Status* v = s;
+  return (v->bad_index | v->timeout) != 0u;
+}
+
 __global__ void __launch_bounds__(kMergeThreads)
 lse_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
                  const float* __restrict__ part_g, int splits, int N,
                  const float* __restrict__ ent, const float* __restrict__ mask,
                  const int32_t* __restrict__ tidx, int Kp, float zscale, float tfac,
-                 float* __restrict__ lse_out, double* __restrict__ term_part) {
+                 float* __restrict__ lse_out, double* __restrict__ term_part,
+                 const Status* poison_on) {
   __shared__ double s_red[kMergeThreads / 32];
   const int n = blockIdx.x * kMergeThreads + threadIdx.x;
   double contrib = 0.0;
-  if (n < N) {
+  if (n < N && status_failed(poison_on)) {
+    lse_out[n] = __int_as_float(0x7fc00000);
+  } else if (n < N) {
     float m = -INFINITY;
     for (int s = 0; s < splits; ++s) m = fmaxf(m, part_m[(size_t)s * N + n]);
     float ssum = 0.f, g = 0.f;
@@ -271,10 +285,13 @@ scatter_rows_kernel(const uint4* __restrict__ src, int d8, const int32_t* __rest
 // Single block.  Sums block partials in a fixed order (deterministic).
 //  mode 0: *loss = sum(term_part) / sum(mask_part), or 0 if the mask sums to 0.
 //  mode 1: *cscale = g / sum(mask_part) (g = *grad or 1), or 0.
+// With `poison_on` set and reporting a failure (see lse_merge_kernel), the
+// output is NaN.
 __global__ void __launch_bounds__(256)
 finalize_kernel(const double* __restrict__ mask_part, int n_mask_part,
                 const double* __restrict__ term_part, int n_term_part, int mode,
-                const float* __restrict__ grad, float* __restrict__ out) {
+                const float* __restrict__ grad, float* __restrict__ out,
+                const Status* poison_on = nullptr) {
   __shared__ double s_m[256], s_t[256];
   double am = 0.0, at = 0.0;
   for (int i = threadIdx.x; i < n_mask_part; i += 256) am += mask_part[i];
@@ -291,7 +308,9 @@ finalize_kernel(const double* __restrict__ mask_part, int n_mask_part,
   }
   if (threadIdx.x == 0) {
     const double sm = s_m[0];
-    if (mode == 0) {
+    if (status_failed(poison_on)) {
+      *out = __int_as_float(0x7fc00000);
+    } else if (mode == 0) {
       *out = (sm != 0.0) ? (float)(s_t[0] / sm) : 0.f;
     } else {
       const double g = grad ? (double)*grad : 1.0;

@@ -19,6 +19,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -79,6 +80,34 @@ Layout make_layout(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   L.off_nrows = take(sizeof(int));
   L.off_hc = take(2 * (size_t)L.C * d);
   L.off_dhc = take(2 * (size_t)L.C * d);
+  L.total = o;
+  return L;
+}
+
+// The regions the forward pass alone uses, at the same offsets rules: status
+// words, scalars, the fp64 block sums, the prepared teacher cache, the
+// per-split (m, s, g) partials and the forward's wave counters.  No dZ
+// chunk, no joint-launch counters, no row map or row buffers.  About
+// 8 Kp + 199 bytes per token, plus under 4 KiB.
+Layout make_forward_layout(int64_t N, int64_t K) {
+  Layout L;
+  L.Kp = (int)round_up(K + 1, 4);
+  L.C = 1;
+  L.n_prep_blocks = ceil_div(N > 0 ? N : 1, kPrepWarps);
+  L.n_merge_blocks = ceil_div(N > 0 ? N : 1, kMergeThreads);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
+  L.off_status = take(sizeof(Status));
+  L.off_scal = take(64);
+  L.off_mask_part = take(sizeof(double) * L.n_prep_blocks);
+  L.off_term_part = take(sizeof(double) * L.n_merge_blocks);
+  L.off_tidx = take(sizeof(int32_t) * (size_t)N * L.Kp);
+  L.off_tp = take(sizeof(float) * (size_t)N * L.Kp);
+  L.off_ent = take(sizeof(float) * (size_t)N);
+  L.off_pm = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_ps = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_pg = take(sizeof(float) * (size_t)N * kMaxSplits);
+  L.off_wave = take(sizeof(unsigned int) * (size_t)wave_slots_bound(ceil_div(N > 0 ? N : 1, 256) * kMaxSplits, 0));
   L.total = o;
   return L;
 }
@@ -317,7 +346,7 @@ struct LaunchEvents {
 int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const Variant& var,
                   const float* mask, int64_t N, int64_t d, int64_t V, int64_t K,
                   const Layout& L, float* loss, float* lse, void* workspace, cudaStream_t s,
-                  LaunchEvents& evs);
+                  LaunchEvents& evs, bool poison = false);
 
 }  // namespace
 
@@ -372,11 +401,13 @@ int kd_topk_kl_forward_ex(const void* H, const void* W, const int32_t* topk_idx,
 namespace {
 
 // Forward pass on a checked workspace layout: clears the status words, then
-// teacher prep, the logits/lse GEMM, the lse merge and the loss.
+// teacher prep, the logits/lse GEMM, the lse merge and the loss.  With
+// `poison`, a bad teacher index or a timed-out wait seen by the pass makes
+// the lse and the loss NaN (for callers that cannot read the status words).
 int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const Variant& var,
                   const float* mask, int64_t N, int64_t d, int64_t V, int64_t K,
                   const Layout& L, float* loss, float* lse, void* workspace, cudaStream_t s,
-                  LaunchEvents& evs) {
+                  LaunchEvents& evs, bool poison) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
 
@@ -429,10 +460,10 @@ int forward_stage(const void* H, const void* W, const int32_t* topk_idx, const V
   if (!evs.mark()) return KD_ERR_CUDA;
   lse_merge_kernel<<<(unsigned)L.n_merge_blocks, kMergeThreads, 0, s>>>(
       ep.part_m, ep.part_s, ep.part_g, a.raster.splits, (int)N, ent, mask, tidx, L.Kp, var.zscale,
-      var.tfac, lse, term_part);
+      var.tfac, lse, term_part, poison ? status : nullptr);
   if (!evs.mark()) return KD_ERR_CUDA;
   finalize_kernel<<<1, 256, 0, s>>>(mask_part, (int)L.n_prep_blocks, term_part,
-                                    (int)L.n_merge_blocks, 0, nullptr, loss);
+                                    (int)L.n_merge_blocks, 0, nullptr, loss, poison ? status : nullptr);
   return cudaGetLastError() == cudaSuccess ? KD_OK : KD_ERR_CUDA;
 }
 
@@ -827,13 +858,18 @@ extern "C" int kd_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
 // fixed scratch array that lives in this library's own device image.
 //
 // The array is kNoAllocScratchBytes (16 MiB) on every device that loads the
-// library and stays allocated until the process exits.  In host code the
-// symbol is only a host-side stand-in, so its device address is looked up
-// with cudaGetSymbolAddress once per device, on that device's first call.
+// library and stays allocated until the process exits.  It holds the
+// forward pass's own regions only (make_forward_layout: about
+// 8 round_up(K + 1, 4) + 199 bytes per token).  In host code the symbol is
+// only a host-side stand-in, so its device address is looked up with
+// cudaGetSymbolAddress once per device, on that device's first call, and
+// kept (an atomic per device, so concurrent first calls from several host
+// threads are benign).  Such a kept address belongs to the device's context
+// of that time: it does not survive cudaDeviceReset.
 
 namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
-void* g_noalloc_scratch_ptr[kMaxDevices] = {};
+std::atomic<void*> g_noalloc_scratch_ptr[kMaxDevices];
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -844,21 +880,29 @@ extern "C" int kd_topk_kl_forward_noalloc(const void* H, const void* W, const in
                                           float* lse, void* stream) {
   int st = check_shapes(N, d, V, K, T, 1);
   if (st != KD_OK) return st;
-  // The forward pass needs no dZ chunk, so the smallest chunk keeps the
-  // layout (and the size limit) to the prepared teacher cache, the per-token
-  // partial log-sum-exp state and the status words.
-  if (make_layout(N, d, V, K, 1).total > kNoAllocScratchBytes) return KD_ERR_WORKSPACE;
+  if (!W || !loss || (N > 0 && (!H || !topk_idx || !topk_logit || !lse))) return KD_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || (H && !aligned(H, 16)) || (topk_idx && !aligned(topk_idx, 4)) ||
+      (topk_logit && !aligned(topk_logit, 4)) || (mask && !aligned(mask, 4)))
+    return KD_ERR_INVALID_ARG;
+  const Layout L = make_forward_layout(N, K);
+  if (L.total > kNoAllocScratchBytes) return KD_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KD_ERR_UNSUPPORTED;
-  if (!g_noalloc_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KD_ERR_CUDA;
-    g_noalloc_scratch_ptr[dev] = p;
+  void* scratch = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!scratch) {
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr)
+      return KD_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev].store(scratch, std::memory_order_release);
   }
-  // Every word the forward pass reads from the scratch is written earlier in
-  // the same call (the status words are cleared at its start), so nothing
-  // left over from a previous call is ever used.
-  return kd_topk_kl_forward(H, W, topk_idx, topk_logit, mask, N, d, V, K, T, 1, loss, lse,
-                            g_noalloc_scratch_ptr[dev], kNoAllocScratchBytes, stream);
+  // Every word the pass reads from the scratch is written earlier in the
+  // same call (the status words are cleared at its start), so nothing left
+  // over from a previous call is used.  The status words cannot be read by
+  // the caller here, so a bad teacher index or a timed-out wait turns the
+  // loss and every lse into NaN instead.
+  Variant var;
+  if ((st = make_variant(nullptr, topk_logit, T, &var)) != KD_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  LaunchEvents evs{nullptr, 0, 0, s};
+  return forward_stage(H, W, topk_idx, var, mask, N, d, V, K, L, loss, lse, scratch, s, evs, true);
 }

@@ -85,6 +85,11 @@ typedef enum kd_status {
   KD_ERR_TIMEOUT = 6       /* (from kd_topk_kl_check) a pipeline wait gave up; results invalid */
 } kd_status;
 
+/* Every entry point returns one of the kd_status values above as a plain
+ * int, not as the enum type: an enum's size is up to the compiler (C allows
+ * a smaller type; -fshort-enums picks one), whereas int is 32 bits for every
+ * caller that binds this library, C or a foreign-function interface. */
+
 /* Human-readable name of a status code.  Never returns NULL. */
 const char* kd_status_string(int status);
 
@@ -168,23 +173,31 @@ int kd_topk_kl_forward_backward(const void* H, const void* W,
  * latency-critical loop that cannot afford cudaMalloc's implicit
  * synchronisation.
  *
- * Same inputs and outputs as kd_topk_kl_forward (no chunk, no workspace).
- * Instead of a caller workspace it uses a 16 MiB scratch array compiled into
- * the library: every device that loads the library holds those 16 MiB until
- * the process exits.  It allocates nothing itself (no cudaMalloc, no
- * cudaFree, no allocating library call).
- *  - Size limit: kd_topk_kl_workspace_size(N, d, V, K, 1) must not exceed
- *    16 MiB (about 1 KiB per token at K = 100, so up to roughly 16,000
- *    tokens); larger sizes return KD_ERR_WORKSPACE and enqueue nothing.
+ * Same inputs and outputs as kd_topk_kl_forward (fp32 logits, no options,
+ * no chunk, no workspace).  Instead of a caller workspace it uses a 16 MiB
+ * scratch array compiled into the library: every device that loads the
+ * library holds those 16 MiB until the process exits.  It allocates nothing
+ * itself (no cudaMalloc, no cudaFree, no allocating library call).
+ *  - Size limit: the scratch holds the forward pass's own state only, about
+ *    8 * round_up(K + 1, 4) + 199 bytes per token plus under 4 KiB.  Sizes
+ *    with (8 * round_up(K + 1, 4) + 199) * N + 4096 <= 16 MiB are accepted
+ *    (N <= 16,268 at K = 100, 46,721 at K = 16), any d and V; sizes with
+ *    (8 * round_up(K + 1, 4) + 198) * N > 16 MiB return KD_ERR_WORKSPACE
+ *    and enqueue nothing.
  *  - The first call on each device looks up the scratch array's device
- *    address (cudaGetSymbolAddress) with that device current; make that
- *    first call before any stream capture begins.
+ *    address (cudaGetSymbolAddress) with that device current and keeps it
+ *    for later calls; make that first call before any stream capture
+ *    begins.  The kept address belongs to the device's context at that
+ *    time and does not survive cudaDeviceReset.
  *  - All calls share the one array and it keeps the last call's contents;
  *    the pass clears its status words and overwrites everything else it
  *    reads before reading it.  Calls that overlap on the GPU (different
  *    streams, or different host threads) race on the array and must not be
- *    issued.  Device-side status (bad teacher indices) is not reported
- *    through kd_topk_kl_check for this entry point. */
+ *    issued.
+ *  - The device-side status words cannot be read by the caller of this
+ *    entry point (kd_topk_kl_check takes a workspace).  Instead, when the
+ *    pass meets a teacher index outside [0, V) or a pipeline wait times
+ *    out, it writes NaN to *loss and to every lse[n]. */
 int kd_topk_kl_forward_noalloc(const void* H, const void* W,
                                const int32_t* topk_idx, const float* topk_logit,
                                const float* mask,

@@ -142,3 +142,29 @@ def test_binding_checks_caller_buffers(lib):
     assert g.shape == () and g.dtype == torch.float32 and float(g) == 2.5
     with pytest.raises(ValueError):
         api._grad_scalar(torch.ones(2), cpu)
+
+
+def test_noalloc_size_limit(lib):
+    """kd_topk_kl_forward_noalloc holds the forward pass's state in a 16 MiB
+    array: the header promises every N with (8 Kp + 199) N + 4096 <= 16 MiB
+    and rejects every N with (8 Kp + 198) N > 16 MiB (Kp = round_up(K+1, 4)),
+    whatever d and V.  Rejection is synchronous, before any CUDA call.  The
+    accepted side is checked only on a machine without a CUDA device, where
+    the call gets past the size check and then fails at cudaGetDevice (with
+    a device it would launch on these fake pointers)."""
+    import math
+    import torch
+    from chunked_top_kl_b200 import _abi
+    P = 1 << 20
+    F = _abi.kd_topk_kl_forward_noalloc
+    no_device = not torch.cuda.is_available()
+    for K in (1, 16, 100, 512):
+        Kp = 4 * math.ceil((K + 1) / 4)
+        n_bad = (16 << 20) // (8 * Kp + 198) + 1
+        n_ok = ((16 << 20) - 4096) // (8 * Kp + 199)
+        for d, V in ((2880, 201088), (8, 64)):
+            assert F(P, P, P, P, None, n_bad, d, V, K, 1.0, P, P, None) == _abi.KD_ERR_WORKSPACE
+            if no_device:
+                assert F(P, P, P, P, None, n_ok, d, V, K, 1.0, P, P, None) == _abi.KD_ERR_CUDA
+    assert F(P, P, P, P, None, 100, 8, 64, 16, 1.0, None, P, None) == _abi.KD_ERR_INVALID_ARG
+    assert F(P, P + 8, P, P, None, 100, 8, 64, 16, 1.0, P, P, None) == _abi.KD_ERR_INVALID_ARG
