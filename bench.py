@@ -280,6 +280,102 @@ def config_block(cfg, world):
             "l2": "inputs larger than L2 (W is %.2f GB > 126 MB L2); no flush" % (2 * cfg.V * cfg.d / 1e9)}
 
 
+def executed_flops(cfg, n_kept=None) -> float:
+    """Tensor-core flops a step runs: the forward GEMM over every token (2NdV)
+    and the backward's three (6 n d V) over the tokens it processes (all, or
+    the kept ones when masked rows are skipped)."""
+    nb = cfg.N if n_kept is None else n_kept
+    return 2.0 * cfg.N * cfg.d * cfg.V + 6.0 * nb * cfg.d * cfg.V
+
+
+def measure_config(kd, cfg, dev, steps: int, warmup: int, backward_rows: str = "auto"):
+    """Device-timed fused steps of one workload on its own inputs (made here,
+    copied to the device before timing, freed after): ms per step, peak HBM
+    GiB of the step over inputs, outputs and workspace, and live per-kernel
+    times.  Used for the secondary workloads of the default run."""
+    x = workloads.make_inputs(cfg)
+    N, d, V, K, T, chunk = cfg.N, cfg.d, cfg.V, cfg.K, cfg.T, cfg.chunk
+    n_kept = int(((x["mask"] != 0) & (x["topk_idx"] != -1).any(dim=1)).sum())
+    skip = backward_rows == "kept" or (backward_rows == "auto" and n_kept < N and N >= AUTO_SKIP_MIN_N)
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_mem = torch.cuda.memory_allocated(dev)
+    g = {k: v.to(dev) for k, v in x.items()}
+    del x
+    ws = kd.alloc_workspace(N, d, V, K, chunk, dev)
+    dH = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nl = kd.forward_backward_launches(N, chunk, skip)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)] for _ in range(steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+
+    def step(events=None):
+        kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], T, chunk,
+                            workspace=ws, dH=dH, dW=dW, events=events, skip_masked_rows=skip)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, _ = kd.check(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up ({cfg.name}): {kd.kd_status_string(st)}")
+    peak_gib = (torch.cuda.max_memory_allocated(dev) - base_mem) / 2**30
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step(ev[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end) / steps
+    kern = per_kernel_times(ev, N, d, V, chunk, n_kept if skip else None)
+    del g, ws, dH, dW
+    torch.cuda.empty_cache()
+    return {"ms": ms, "peak_gib": peak_gib, "kern": kern, "n_kept": n_kept if skip else None}
+
+
+def secondary_block(kd, dev, args, peaks):
+    """The other workloads on which the target is stated, measured in the
+    same run: the Llama-shaped 8K head (V = 128,256) and every point of the
+    long-context sweep (d = 2048, V = 128,256, 4K to 256K tokens) with its
+    peak HBM and a least-squares line through peak GiB against N."""
+    out = {}
+    peak, peak_sus = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+
+    def entry(cfg, r):
+        tf = 8.0 * cfg.N * cfg.d * cfg.V / (r["ms"] / 1e3) / 1e12
+        tfx = executed_flops(cfg, r["n_kept"]) / (r["ms"] / 1e3) / 1e12
+        dom = max((v for v in r["kern"].values() if v["flops"] > 0), key=lambda v: v["ms"])
+        return {"N": cfg.N, "d": cfg.d, "V": cfg.V, "chunk": cfg.chunk, "ms_per_step": r["ms"],
+                "tokens_per_s": cfg.N / (r["ms"] / 1e3), "tflops": tf, "tflops_executed": tfx,
+                "pct_bf16_peak": tf / peak, "pct_bf16_peak_sustained": tf / peak_sus,
+                "peak_hbm_gib": r["peak_gib"],
+                "kernel_tflops": {k: v["tflops"] for k, v in r["kern"].items() if v["tflops"]},
+                "dominant_kernel_frac_sustained": dom["tflops"] / peak_sus}
+
+    cfg2 = workloads.get_config(2)
+    out[cfg2.name] = entry(cfg2, measure_config(kd, cfg2, dev, args.secondary_steps, 3))
+    sweep = []
+    cfg4 = workloads.get_config(4)
+    for n in cfg4.sweep:
+        c = workloads.get_config(4, n)
+        sweep.append(entry(c, measure_config(kd, c, dev, args.secondary_steps, 3)))
+    ns = [e["N"] for e in sweep]
+    gib = [e["peak_hbm_gib"] for e in sweep]
+    mn, mg = sum(ns) / len(ns), sum(gib) / len(gib)
+    slope = sum((a - mn) * (b - mg) for a, b in zip(ns, gib)) / sum((a - mn) ** 2 for a in ns)
+    icpt = mg - slope * mn
+    resid = max(abs(b - (icpt + slope * a)) / b for a, b in zip(ns, gib))
+    out[cfg4.name] = {"points": sweep,
+                      "peak_gib_fit": {"slope_bytes_per_token": slope * 2**30, "intercept_gib": icpt,
+                                       "max_rel_residual": resid}}
+    return out
+
+
 def run_cuda(args, cfg, world, rank, local):
     import chunked_top_kl_b200 as kd
 
@@ -414,7 +510,10 @@ def run_cuda(args, cfg, world, rank, local):
         e2e = {"value": N * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(loss_host.element_size()),
                "ms_per_step": e2e_ms / args.steps,
-               "copies": "step k+1's inputs copied on a second stream during step k (two device input sets)",
+               "copies": ("every input (H, W, teacher cache, mask) copied in from pinned host memory each "
+                          "step, step k+1's on a second stream during step k (two device input sets); "
+                          "only the loss is read back: dH and dW stay on the device for the optimizer, "
+                          "as in a training step"),
                "serial_ms_per_step": serial_ms / args.steps}
         del g2
 
@@ -422,9 +521,15 @@ def run_cuda(args, cfg, world, rank, local):
         return 0
 
     peaks, peaks_src = load_peaks()
+    secondary = None
+    if world == 1 and not args.no_secondary:
+        del g, ws, dH, dW
+        torch.cuda.empty_cache()
+        secondary = secondary_block(kd, dev, args, peaks)
     ms_step = ms / args.steps
     flops_step = 8.0 * N * d * V
     tflops = flops_step * world / (ms_step / 1e3) / 1e12
+    tflops_exec = executed_flops(cfg, kept) * world / (ms_step / 1e3) / 1e12
     # Roofline of the dominant kernel (largest share of the step's kernel time).
     dom_name, dom = max(((k, v) for k, v in kern.items() if v["flops"] > 0), key=lambda kv: kv[1]["ms"])
     dom_ach = dom["tflops"]
@@ -446,6 +551,11 @@ def run_cuda(args, cfg, world, rank, local):
         "tflops": tflops,
         "pct_bf16_peak": tflops / world / peaks["bf16_tflops"],
         "pct_bf16_peak_sustained": tflops / world / peak_sus,
+        "tflops_executed": tflops_exec,
+        "pct_bf16_peak_executed": tflops_exec / world / peaks["bf16_tflops"],
+        "flops_note": ("tflops counts 8 N d V per step (the metric's count); tflops_executed counts the "
+                       "tensor-core work the step runs (2 N d V forward + 6 n d V backward over the "
+                       "n tokens it processes)"),
         "peak_hbm_gib": peak_gib, "workspace_gib": ws_gib,
         "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
         "config": {**config_block(cfg, world), "backward_rows": "kept tokens only" if skip else "all tokens"},
@@ -464,6 +574,7 @@ def run_cuda(args, cfg, world, rank, local):
                           "flops_per_step": flops_step},
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "secondary": secondary,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -588,6 +699,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the Llama-shaped head and the long-context sweep measured after the main workload")
+    ap.add_argument("--secondary-steps", type=int, default=5, help="timed steps per secondary workload")
     ap.add_argument("--backward-rows", choices=["auto", "all", "kept"], default="auto",
                     help="backward over every token, or over the tokens with a non-zero dZ row only "
                          "(same results; auto: kept when some token is masked and N >= %d)" % AUTO_SKIP_MIN_N)
