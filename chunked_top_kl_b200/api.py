@@ -78,6 +78,14 @@ def alloc_workspace(N, d, V, K, chunk, device) -> torch.Tensor:
     return torch.empty(workspace_bytes(N, d, V, K, chunk), dtype=torch.uint8, device=device)
 
 
+def _on(dev):
+    """The library works on the calling thread's current CUDA device (its
+    occupancy figures, tensor maps and the no-allocation scratch address
+    come from cudaGetDevice), so every call is made with the inputs' device
+    current."""
+    return torch.cuda.device(dev)
+
+
 def _raise(st: int, where: str):
     if st != _abi.KD_OK:
         raise _abi.KDError(st, where)
@@ -120,16 +128,18 @@ def forward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chunk: int = 
     lse = torch.empty(N, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     opt = _options(topk_logit, student_temperature)
-    if opt is None:
-        st = _abi.kd_topk_kl_forward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
-                                     N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
-                                     _ptr(workspace), workspace.numel(), stream)
-        _raise(st, "kd_topk_kl_forward")
-    else:
-        st = _abi.kd_topk_kl_forward_ex(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
-                                        N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
-                                        _ptr(workspace), workspace.numel(), stream, opt)
-        _raise(st, "kd_topk_kl_forward_ex")
+    with _on(dev):
+        if opt is None:
+            st = _abi.kd_topk_kl_forward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                         N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
+                                         _ptr(workspace), workspace.numel(), stream)
+            where = "kd_topk_kl_forward"
+        else:
+            st = _abi.kd_topk_kl_forward_ex(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                            N, d, V, K, float(T), int(chunk), _ptr(loss), _ptr(lse),
+                                            _ptr(workspace), workspace.numel(), stream, opt)
+            where = "kd_topk_kl_forward_ex"
+    _raise(st, where)
     return loss, lse
 
 
@@ -166,25 +176,27 @@ def backward(H, W, topk_idx, topk_logit, mask, T: float, chunk: int, lse: torch.
     grad_loss = _grad_scalar(grad_loss, dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     opt = _options(topk_logit, student_temperature, skip_masked_rows)
-    if opt is not None:
-        st = _abi.kd_topk_kl_backward_ex(
-            _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
-            int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
-            _ptr(workspace), workspace.numel(), stream,
-            _event_handles(events), opt)
-        _raise(st, "kd_topk_kl_backward_ex")
-    elif events is None:
-        st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
-                                      N, d, V, K, float(T), int(chunk), _ptr(lse), _ptr(grad_loss),
-                                      _ptr(dH), _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
-                                      workspace.numel(), stream)
-        _raise(st, "kd_topk_kl_backward")
-    else:
-        st = _abi.kd_topk_kl_backward_profiled(
-            _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
-            int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
-            _ptr(workspace), workspace.numel(), stream, _event_handles(events))
-        _raise(st, "kd_topk_kl_backward_profiled")
+    evs = _event_handles(events)
+    with _on(dev):
+        if opt is not None:
+            st = _abi.kd_topk_kl_backward_ex(
+                _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
+                int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+                _ptr(workspace), workspace.numel(), stream, evs, opt)
+            where = "kd_topk_kl_backward_ex"
+        elif events is None:
+            st = _abi.kd_topk_kl_backward(_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask),
+                                          N, d, V, K, float(T), int(chunk), _ptr(lse), _ptr(grad_loss),
+                                          _ptr(dH), _ptr(dW), int(bool(accumulate_dW)), _ptr(workspace),
+                                          workspace.numel(), stream)
+            where = "kd_topk_kl_backward"
+        else:
+            st = _abi.kd_topk_kl_backward_profiled(
+                _ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T),
+                int(chunk), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
+                _ptr(workspace), workspace.numel(), stream, evs)
+            where = "kd_topk_kl_backward_profiled"
+    _raise(st, where)
     return dH, dW
 
 
@@ -221,10 +233,12 @@ def forward_backward(H, W, topk_idx, topk_logit, mask=None, T: float = 1.0, chun
     args = (_ptr(H), _ptr(W), _ptr(topk_idx), _ptr(topk_logit), _ptr(mask), N, d, V, K, float(T), int(chunk),
             _ptr(loss), _ptr(lse), _ptr(grad_loss), _ptr(dH), _ptr(dW), int(bool(accumulate_dW)),
             _ptr(workspace), workspace.numel(), stream)
-    if opt is None:
-        _raise(_abi.kd_topk_kl_forward_backward(*args, evs), "kd_topk_kl_forward_backward")
-    else:
-        _raise(_abi.kd_topk_kl_forward_backward_ex(*args, evs, opt), "kd_topk_kl_forward_backward_ex")
+    with _on(dev):
+        if opt is None:
+            st, where = _abi.kd_topk_kl_forward_backward(*args, evs), "kd_topk_kl_forward_backward"
+        else:
+            st, where = _abi.kd_topk_kl_forward_backward_ex(*args, evs, opt), "kd_topk_kl_forward_backward_ex"
+    _raise(st, where)
     return loss, lse, dH, dW
 
 
@@ -251,8 +265,9 @@ def teacher_topk(Ht, Wt, K: int, chunk: int = 1024,
     idx = torch.empty((N, K), dtype=torch.int32, device=dev)
     val = torch.empty((N, K), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    st = _abi.kd_teacher_topk(_ptr(Ht), _ptr(Wt), N, d, V, int(K), int(chunk), _ptr(idx), _ptr(val),
-                              _ptr(workspace), workspace.numel(), stream)
+    with _on(dev):
+        st = _abi.kd_teacher_topk(_ptr(Ht), _ptr(Wt), N, d, V, int(K), int(chunk), _ptr(idx), _ptr(val),
+                                  _ptr(workspace), workspace.numel(), stream)
     _raise(st, "kd_teacher_topk")
     return idx, val
 
@@ -261,7 +276,8 @@ def check(workspace: torch.Tensor) -> Tuple[int, int]:
     """Synchronise the current stream and read the device status words:
     returns (status, bad_index_count)."""
     stream = torch.cuda.current_stream(workspace.device).cuda_stream
-    return _abi.kd_topk_kl_check(_ptr(workspace), stream)
+    with _on(workspace.device):
+        return _abi.kd_topk_kl_check(_ptr(workspace), stream)
 
 
 class KDTopKKLFunction(torch.autograd.Function):

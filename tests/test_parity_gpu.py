@@ -91,8 +91,11 @@ SMALL_CASES = [
     (1, 64, 24, 5, 2.0, 4096, "ones"),                # single token, V < one tile
     (700, 512, 5000, 100, 1.3, 256, "drop5"),         # K = 100, many tiles
     (256, 8, 300, 300, 1.0, 128, "ones"),             # K = V (whole vocabulary), d = 8
-    (300, 320, 2000, 12, 1.1, 128, "drop5"),          # d = 256 + 64: a narrow last column tile of dH / dW
-    (260, 384, 1500, 9, 1.0, 128, "ones"),            # d = 256 + 128: a last column tile exactly half wide
+    (300, 320, 2000, 12, 1.1, 128, "drop5"),          # d = 2 x 160: dH / dW tiles narrower than 256, dH tail of 32
+    (260, 384, 1500, 9, 1.0, 128, "ones"),            # d = 2 x 192: narrow tiles, whole 64-column boxes
+    (300, 240, 2000, 12, 1.0, 96, "drop5"),           # d = 240: one tile, dH tail of 48 and dW tail of 16 columns
+    (520, 480, 3000, 20, 0.9, 256, "ones"),           # d = 2 x 240 (the 2880 = 12 x 240 split in small)
+    (200, 136, 900, 10, 1.0, 64, "ones"),             # d = 136: no equal split, a 256 tile clipped at d
 ]
 
 
@@ -172,12 +175,14 @@ def test_neg_inf_teacher_logit(kd):
     _assert_parity(got, ref, "-inf logits")
 
 
-def test_accumulate_dW(kd):
-    x = workloads.make_inputs(_cfg(200, 64, 700, 6, seed=8))
+@pytest.mark.parametrize("d", [64, 240])
+def test_accumulate_dW(kd, d):
+    # d = 240: the last 16 columns of each dW tile are added from registers
+    x = workloads.make_inputs(_cfg(200, d, 700, 6, seed=8))
     g = _to_dev(x)
-    ws = kd.alloc_workspace(200, 64, 700, 6, 64, "cuda")
+    ws = kd.alloc_workspace(200, d, 700, 6, 64, "cuda")
     _, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, workspace=ws)
-    dW0 = torch.randn(700, 64, device="cuda")
+    dW0 = torch.randn(700, d, device="cuda")
     _, dW = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, lse,
                         dW=dW0.clone(), accumulate_dW=True, workspace=ws)
     _, dW1 = kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 64, lse,
@@ -290,3 +295,27 @@ def test_caller_buffers_are_checked(kd):
     torch.cuda.synchronize()
     dH, dW = kd.backward(*args, lse, workspace=ws)     # the same call with valid buffers still runs
     assert kd.check(ws) == (0, 0) and torch.isfinite(dW).all()
+
+
+def test_calls_run_with_the_inputs_device_current(kd, monkeypatch):
+    """The library reads the device from cudaGetDevice, so the binding makes
+    the inputs' device current around every call."""
+    from chunked_top_kl_b200 import api
+    seen = []
+    real = api._on
+
+    def spy(dev):
+        seen.append(torch.device(dev))
+        return real(dev)
+
+    monkeypatch.setattr(api, "_on", spy)
+    x = workloads.make_inputs(_cfg(64, 64, 500, 8, seed=11))
+    g = _to_dev(x)
+    ws = kd.alloc_workspace(64, 64, 500, 8, 32, g["H"].device)
+    loss, lse = kd.forward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 32, workspace=ws)
+    kd.backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 32, lse, workspace=ws)
+    kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, 32, workspace=ws)
+    kd.teacher_topk(g["H"], g["W"], 8, chunk=32)
+    st, _ = kd.check(ws)
+    assert st == 0
+    assert len(seen) == 5 and all(d == g["H"].device for d in seen), seen
