@@ -157,18 +157,20 @@ def _masked_inputs(N, d, V, K, seed, frac):
     return x
 
 
-@pytest.mark.parametrize("frac,chunk", [(0.05, 128), (0.6, 64), (1.0, 96)], ids=["drop5", "drop60", "all"])
-def test_skip_masked_rows(kd, frac, chunk):
+@pytest.mark.parametrize("frac,chunk,d", [(0.05, 128, 136), (0.6, 64, 136), (1.0, 96, 136), (0.05, 128, 240),
+                                          (1.0, 96, 240)],
+                         ids=["drop5", "drop60", "all", "drop5_d240", "all_d240"])
+def test_skip_masked_rows(kd, frac, chunk, d):
     # the backward over the kept tokens only: the forward is untouched, dH
     # equal bit for bit (every dZ row is computed the same way), dW equal up
     # to the fp32 order of the chunk sums; with 60 % dropped the trailing
     # chunks have no live row, with everything dropped dW must still be zeroed
-    x = _masked_inputs(700, 136, 3000, 24, seed=44, frac=frac)
+    x = _masked_inputs(700, d, 3000, 24, seed=44, frac=frac)
     x["topk_idx"] = _empty_slots(x["topk_idx"], 44, frac=0.1, empty_rows=(3,))
     a = _run(kd, x, 1.0, chunk, grad=1.4, student_temperature=False)
     g = {k: v.cuda() for k, v in x.items()}
-    ws = kd.alloc_workspace(700, 136, 3000, 24, chunk, "cuda")
-    dW = torch.full((3000, 136), float("nan"), device="cuda")     # overwritten, never read
+    ws = kd.alloc_workspace(700, d, 3000, 24, chunk, "cuda")
+    dW = torch.full((3000, d), float("nan"), device="cuda")       # overwritten, never read
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(kd.forward_backward_launches(700, chunk, True) + 1)]
     for e in evs:
         e.record()                       # creates the CUDA event behind each object
