@@ -117,7 +117,7 @@ __device__ __forceinline__ void apply_live_rows(GemmArgs& a, int rows, int ngrou
     if (pa.dyn_role == 1) {
       pa.raster = tile_raster(ceil_div64(rows, G::TILE_M), pa.raster.n_tiles, pa.dyn_bands_fastest != 0);
     } else if (pa.dyn_role == 3) {
-      pa.raster = forward_raster(ceil_div64(rows, G::TILE_M), pa.raster.n_tiles, ngroups);
+      pa.raster = forward_raster(ceil_div64(rows, G::TILE_M), pa.raster.n_tiles, ngroups, 0, 0, kMaxDzSplits);
     } else if (pa.dyn_role == 2) {
       pa.num_kb = (int)ceil_div64(rows, BK);
       if (rows == 0 && !pa.dyn_zero_fill) pa.raster.num_units = 0;

@@ -13,7 +13,8 @@
 
 namespace kd {
 
-constexpr int kMaxSplits = 16;   // column ranges per band in the forward pass
+constexpr int kMaxSplits = 16;   // column ranges per band in the forward pass (its partials)
+constexpr int kMaxDzSplits = 64; // column ranges per band in the dZ recompute (no partials)
 
 KD_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -61,9 +62,13 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
 
 // Forward pass (and the dZ recompute): a unit is a band and a range of
 // vocabulary tiles whose running log-sum-exp (or teacher-column cursor) one
-// CTA carries.  Picks the number of ranges
-// (<= kMaxSplits) minimising waves x longest range on `grid` CTAs; every
-// range is non-empty.
+// CTA carries.  Picks the number of ranges (<= max_splits; every range is
+// non-empty) that minimises the tiles of the busiest of `grid` CTAs.  Units
+// go round-robin and the longer ranges (n_tiles % S of them, one tile
+// longer) come first in the unit order, so CTA 0 has both the most units,
+// w = ceil(m S / grid), and the most long ones, ceil(m (n_tiles % S) / grid)
+// at most: its load is w (n_tiles / S) + min(w, that).  (Exact for one band
+// group, and it picks the best S for the grouped forward rasters too.)
 //
 // The B operand (the vocabulary rows) is the large one, so a wave should
 // share each column tile among as many bands as it can: group_m bands walk
@@ -71,11 +76,13 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
 // capped so the group's A bands (band_bytes each, kept in L2) take at most
 // half of `l2_budget`, and evened out over the groups.
 KD_HD Raster forward_raster(int64_t m_tiles, int64_t n_tiles, int grid, int64_t band_bytes = 0,
-                            int64_t l2_budget = 0) {
+                            int64_t l2_budget = 0, int max_splits = kMaxSplits) {
   int best_s = 1;
   int64_t best_cost = (int64_t)1 << 62;
-  for (int s = 1; s <= kMaxSplits && s <= n_tiles; ++s) {
-    const int64_t cost = ceil_div64(m_tiles * s, grid) * ceil_div64(n_tiles, s);
+  for (int s = 1; s <= max_splits && s <= n_tiles; ++s) {
+    const int64_t w = ceil_div64(m_tiles * s, grid);
+    const int64_t longs = ceil_div64(m_tiles * (n_tiles % s), grid);
+    const int64_t cost = w * (n_tiles / s) + (longs < w ? longs : w);
     if (cost < best_cost) { best_cost = cost; best_s = s; }
   }
   Raster r;

@@ -567,7 +567,7 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     // Units are a band and a range of column tiles, so each epilogue thread
     // sets up its token (scale, lse, teacher cursor) once per unit.
     ProbArgs a3{};
-    a3.raster = forward_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), groups);
+    a3.raster = forward_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), groups, 0, 0, kMaxDzSplits);
     a3.num_kb = (int)ceil_div(d, BK);
     a3.a_row0 = hrow0;
     a3.dyn_role = 3;
@@ -786,6 +786,7 @@ int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_
   if (N == 0) return KD_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KD_ERR_UNSUPPORTED;
   float* zbuf = at<float>(workspace, L.off_z);
 
   CUtensorMap tmH, tmW;

@@ -41,7 +41,11 @@ int main() {
           if (r.splits > kMaxSplits) { printf("FAIL splits %d\n", r.splits); return 1; }
           if (r.group_m < 1 || r.group_m > r.m_tiles) { printf("FAIL group_m\n"); return 1; }
           if (!check(r, "fwd", N, V, g)) return 1;
-          ++cases;
+          // the dZ recompute's raster: more ranges allowed, no band groups capped by L2
+          Raster rz = forward_raster(ceil_div64(N, 128), ceil_div64(V, 256), g, 0, 0, kMaxDzSplits);
+          if (rz.splits > kMaxDzSplits) { printf("FAIL dz splits %d\n", rz.splits); return 1; }
+          if (!check(rz, "dzr", N, V, g)) return 1;
+          cases += 2;
         }
   for (long C : chunks)
     for (long V : Vs)
