@@ -696,6 +696,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
     ap.add_argument("--N", type=int, default=None, help="override the token count (config 4 sweep)")
+    ap.add_argument("--V", type=int, default=None, help="override the vocabulary (a smaller case to profile)")
+    ap.add_argument("--d", type=int, default=None, help="override the hidden size (a smaller case to profile)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -717,6 +719,11 @@ def main(argv=None):
     if args.op == "teacher-topk" and args.impl == "reference":
         ap.error("--op teacher-topk times the library; its oracle is timed in cpu_baseline")
     cfg = workloads.get_config(args.config, args.N)
+    if args.V is not None or args.d is not None:
+        import dataclasses
+        V = args.V if args.V is not None else cfg.V
+        d = args.d if args.d is not None else cfg.d
+        cfg = dataclasses.replace(cfg, V=V, d=d, name=f"{cfg.name}_at_N{cfg.N}_d{d}_V{V}")
     world, rank, local = dist_setup(args.impl)
     if world != args.gpus and args.impl == "cuda":
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)

@@ -3,29 +3,50 @@
 // equal values in increasing column order (the order in which an offline
 // cache lists a position's top-K teacher logits).
 //
-// One CTA per row, values mapped to order-preserving 32-bit keys.  A first
-// pass over the row (16-byte loads, four in flight per thread) builds a
-// histogram of the top 12 key bits, which gives the bin holding the K-th
-// largest value and the number of values in or above that bin.  Usually
-// that is a few hundred at most: a second pass copies them into shared
-// memory as (key, column) pairs and a bitonic sort orders them exactly, so
-// the row is read twice.  When the bin is too full (heavily tied rows) the
-// select continues as a radix select instead: two more histogram passes
-// (12 + 8 bits) over the values matching the key prefix found so far, a
-// collection pass that takes every value above the K-th and, of those
-// equal to it, the ones with the lowest column indices (threads own
-// contiguous column ranges, so a scan of per-thread counts orders them),
-// and the same sort of the K pairs.
+// One CTA per row, values mapped to order-preserving 32-bit keys, and one
+// read of the row.  The threads stream the row with 16-byte loads (kSelVec of
+// them in flight per thread, consecutive threads on consecutive addresses),
+// and a value becomes a candidate, appended to a shared-memory list, when
+// its key is at least the current threshold tau.  tau is always the K-th
+// largest key among a subset of the values seen so far, so a value below it
+// is beaten by K others and can never be in the top K, while every value at
+// or above the final tau is on the list.  The first block of the row sets tau
+// to the smallest, over the warps, of each warp's ceil(K/8)-th largest lane
+// maximum (each warp then holds that many distinct values at or above it),
+// and then to the exact K-th largest key of the list; after every kSelSegment
+// blocks the threads meet, and when the list has grown past a quarter of its
+// capacity tau is raised to the exact K-th largest key of the list by a radix
+// select over shared memory and the list is compacted.  A thread first
+// compares the maximum of its values with tau in floats and only then looks
+// at single values, so after the first blocks a value costs a load and a max.
+// At the end the list is cut to the keys at or above its K-th largest and
+// sorted by (key desc, column asc).
+//
+// For logits in no particular order the list stays small.  Rows where it
+// overflows (more candidates in one segment than the list holds: values
+// rising along the row, or heavy ties) are selected by the exact fallback
+// below, which reads the row again: a histogram of the top 12 key bits
+// locates the bin of the K-th largest value; when the values in or above it
+// fit the sort buffer they are copied and sorted, otherwise a radix select
+// (12 + 8 more bits) finds the K-th largest key and a collection pass takes
+// every value above it and, of those equal to it, the ones with the lowest
+// column indices (threads own contiguous column ranges, so a scan of
+// per-thread counts orders them).
 #pragma once
 
 #include <cstdint>
 #include <cuda_runtime.h>
 
+
 namespace kd {
 
 constexpr int kSelectThreads = 256;
 constexpr int kMaxTopK = 512;
-constexpr int kCandCap = 2048;       // candidates sorted in shared memory (power of two, >= kMaxTopK)
+constexpr int kSelVec = 8;           // float4 loads per thread per block of the row
+constexpr int kSelBlock = kSelectThreads * kSelVec;   // float4s per block (8192 values)
+constexpr int kSelSegment = 4;       // blocks between two meetings of the threads
+constexpr int kSelCap = 2048;        // candidate list (power of two, >= 2 kMaxTopK)
+constexpr int kCandCap = 2048;       // fallback sort buffer (power of two, >= kMaxTopK)
 
 // Order-preserving map of a float onto uint32 (larger float, larger key).
 __device__ __forceinline__ uint32_t float_key(float v) {
@@ -37,6 +58,13 @@ __device__ __forceinline__ uint32_t float_key(float v) {
 __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
+
+// A (key, column) pair as one sortable word: larger key first, then lower column.
+__device__ __forceinline__ unsigned long long pack_pair(uint32_t k, int v) {
+  return ((unsigned long long)k << 32) | (unsigned long long)(0xffffffffu - (uint32_t)v);
+}
+
+__device__ __forceinline__ uint32_t pair_key(unsigned long long e) { return (uint32_t)(e >> 32); }
 
 // Block-wide exclusive scan of one int per thread (kSelectThreads threads).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int* total) {
@@ -53,6 +81,140 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int* tota
   *total = s_tmp[kSelectThreads - 1];
   __syncthreads();
   return incl - v;
+}
+
+// Descending bitonic sort of s[0, P), P a power of two (all threads).
+__device__ __forceinline__ void bitonic_sort_desc(unsigned long long* s, int P) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < P; i += kSelectThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const unsigned long long a = s[i], b = s[j];
+          if (desc ? (a < b) : (a > b)) {
+            s[i] = b;
+            s[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Shared state of the selection of one row.  The fallback sorts in the
+// candidate list (its first kCandCap entries) and keeps its own histogram.
+struct SelShared {
+  unsigned long long list[kSelCap];     // candidates (key, column)
+  int fhist[4096];                      // the fallback's histogram
+  int hist[256];                        // radix histogram of the streaming route
+  int scan[kSelectThreads];
+  uint32_t wkey[kSelectThreads / 32];
+  int count, found, need, ncand, over_flag;
+  uint32_t prefix, mask;
+};
+static_assert(kCandCap <= kSelCap, "the fallback sorts in the candidate list");
+
+__device__ __forceinline__ unsigned long long* fallback_sort(SelShared& S) { return S.list; }
+__device__ __forceinline__ int* fallback_hist(SelShared& S) { return S.fhist; }
+
+// Warp 0: finds, in the 256-bin histogram, the highest bin b whose suffix sum
+// (bins b..255) reaches `need`, and writes S.prefix = prefix | b << sh and
+// S.need = the count still needed inside bin b.  Lane l owns bins 8l..8l+7.
+// With fewer than `need` values in all (not reached by the callers) bin 0.
+__device__ __forceinline__ void suffix_bin(SelShared& S, int need, uint32_t prefix, int sh) {
+  const int lane = threadIdx.x & 31;
+  int c[8], own = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = S.hist[8 * lane + i];
+    own += c[i];
+  }
+  int suf = own;                          // inclusive suffix sum over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += x;
+  }
+  const int above = suf - own;
+  const bool mine = above < need && suf >= need;
+  if (mine) {
+    int acc = above, b = 8 * lane;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      if (acc + c[i] >= need) { b = 8 * lane + i; break; }
+      acc += c[i];
+    }
+    S.prefix = prefix | ((uint32_t)b << sh);
+    S.need = need - acc;
+  }
+  if (__ballot_sync(0xffffffffu, mine) == 0u && lane == 0) {
+    S.prefix = prefix;
+    S.need = need;
+  }
+}
+
+// Adds 1 to hist[bin] for every lane with `pred`, one shared atomic per
+// distinct bin of the warp (all 32 lanes call it together).
+__device__ __forceinline__ void warp_hist_add(int* hist, bool pred, uint32_t bin) {
+  const uint32_t b = pred ? bin : 0xffffffffu;
+  const unsigned peers = __match_any_sync(0xffffffffu, b);
+  if (pred && (threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+}
+
+// Exact K-th largest key among list[0, n) (n >= K).  Radix select, 4 passes
+// of 8 bits.  All threads call it.
+__device__ __forceinline__ uint32_t kth_key(SelShared& S, int n, int K) {
+  const int t = threadIdx.x;
+  const int lane = t & 31, w = t >> 5;
+  uint32_t prefix = 0u, pmask = 0u;
+  int need = K;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int sh = 24 - 8 * pass;
+    S.hist[t] = 0;
+    __syncthreads();
+    for (int base = 32 * w; base < n; base += kSelectThreads) {     // warp-uniform trip count
+      const int i = base + lane;
+      const uint32_t k = i < n ? pair_key(S.list[i]) : 0u;
+      warp_hist_add(S.hist, i < n && (k & pmask) == prefix, (k >> sh) & 255u);
+    }
+    __syncthreads();
+    if (t < 32) suffix_bin(S, need, prefix, sh);
+    __syncthreads();
+    prefix = S.prefix;
+    need = S.need;
+    pmask |= 255u << sh;
+  }
+  return prefix;
+}
+
+// Keeps the entries of list[0, n) whose key is >= tau (order not kept);
+// returns the new count.  Each thread reads its kSelCap / kSelectThreads
+// entries into registers before any is written.  All threads call it.
+__device__ __forceinline__ int compact_list(SelShared& S, int n, uint32_t tau) {
+  constexpr int kPer = kSelCap / kSelectThreads;
+  const int t = threadIdx.x;
+  unsigned long long e[kPer];
+  uint32_t keep = 0u;
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int j = t * kPer + i;
+    e[i] = j < n ? S.list[j] : 0ull;
+    if (j < n && pair_key(e[i]) >= tau) {
+      keep |= 1u << i;
+      ++c;
+    }
+  }
+  int total;
+  int o = block_exclusive_scan(c, S.scan, &total);    // its barriers order every read before the writes
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    if (keep & (1u << i)) S.list[o++] = e[i];
+  __syncthreads();
+  return total;
 }
 
 // Calls f(v, value) for every column v < V of a row (16-byte aligned): four
@@ -86,73 +248,37 @@ __device__ __forceinline__ void for_each_value(const float* __restrict__ row, in
   for (int v = 4 * V4 + t; v < V; v += kSelectThreads) f(v, row[v]);
 }
 
-// A (key, column) pair as one sortable word: larger key first, then lower column.
-__device__ __forceinline__ unsigned long long pack_pair(uint32_t k, int v) {
-  return ((unsigned long long)k << 32) | (unsigned long long)(0xffffffffu - (uint32_t)v);
-}
-
-// Descending bitonic sort of s[0, P), P a power of two (all threads).
-__device__ __forceinline__ void bitonic_sort_desc(unsigned long long* s, int P) {
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < P; i += kSelectThreads) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool desc = (i & size) == 0;
-          const unsigned long long a = s[i], b = s[j];
-          if (desc ? (a < b) : (a > b)) {
-            s[i] = b;
-            s[j] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-}
-
-// z: rows of `ldz` fp32 values (ldz a multiple of 4, rows 16-byte aligned),
-// the first V of each valid.  Writes K int32 indices and K fp32 logits per
-// row to idx_out / val_out (row r at out_row0 + r, K per row).
-__global__ void __launch_bounds__(kSelectThreads)
-topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int out_row0,
-                   int32_t* __restrict__ idx_out, float* __restrict__ val_out) {
-  __shared__ int s_hist[4096];
-  __shared__ int s_scan[kSelectThreads];
-  __shared__ unsigned long long s_sort[kCandCap];
-  __shared__ int s_found, s_ncand;
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_need;
-
+// The exact fallback (see the file comment), reading the row from global
+// memory; leaves the K results first in fallback_sort(S).
+__device__ __forceinline__ void select_two_pass(SelShared& S, const float* __restrict__ row, int V, int K) {
   const int t = threadIdx.x;
-  const float* row = z + (size_t)blockIdx.x * ldz;
-
+  unsigned long long* s_sort = fallback_sort(S);
+  int* fh = fallback_hist(S);
   // pass 1: histogram of the top 12 key bits over the whole row
-  for (int b = t; b < 4096; b += kSelectThreads) s_hist[b] = 0;
-  if (t == 0) s_found = 0;
+  for (int b = t; b < 4096; b += kSelectThreads) fh[b] = 0;
+  if (t == 0) S.found = 0;
   __syncthreads();
-  for_each_value(row, V, [&](int, float x) { atomicAdd(&s_hist[float_key(x) >> 20], 1); });
+  for_each_value(row, V, [&](int, float x) { atomicAdd(&fh[float_key(x) >> 20], 1); });
   __syncthreads();
   if (t == 0) {
-    // walk the bins from the top until K values are covered
     int need = K, b = 4095;
-    for (; b > 0 && s_hist[b] < need; --b) need -= s_hist[b];
-    s_need = need;                          // values of bin b still to take
-    s_prefix = (uint32_t)b << 20;
-    s_mask = 0xfff00000u;
-    s_ncand = K - need + s_hist[b];         // values with key >= b << 20
+    for (; b > 0 && fh[b] < need; --b) need -= fh[b];
+    S.need = need;                          // values of bin b still to take
+    S.prefix = (uint32_t)b << 20;
+    S.mask = 0xfff00000u;
+    S.ncand = K - need + fh[b];             // values with key >= b << 20
   }
   __syncthreads();
-  const int ncand = s_ncand;
+  const int ncand = S.ncand;
 
   int P = 1;
   if (ncand <= kCandCap) {
     // pass 2: every value in or above the K-th value's bin, sorted exactly
-    const uint32_t lo = s_prefix;
+    const uint32_t lo = S.prefix;
     for_each_value(row, V, [&](int v, float x) {
       const uint32_t k = float_key(x);
       if (k >= lo) {
-        const int slot = atomicAdd(&s_found, 1);
+        const int slot = atomicAdd(&S.found, 1);
         if (slot < kCandCap) s_sort[slot] = pack_pair(k, v);
       }
     });
@@ -168,25 +294,25 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
     for (int pass = 0; pass < 2; ++pass) {
       const int sh = shifts[pass];
       const int nb = 1 << widths[pass];
-      for (int b = t; b < nb; b += kSelectThreads) s_hist[b] = 0;
+      for (int b = t; b < nb; b += kSelectThreads) fh[b] = 0;
       __syncthreads();
-      const uint32_t prefix = s_prefix, mask = s_mask;
+      const uint32_t prefix = S.prefix, mask = S.mask;
       for_each_value(row, V, [&](int, float x) {
         const uint32_t k = float_key(x);
-        if ((k & mask) == prefix) atomicAdd(&s_hist[(k >> sh) & (uint32_t)(nb - 1)], 1);
+        if ((k & mask) == prefix) atomicAdd(&fh[(k >> sh) & (uint32_t)(nb - 1)], 1);
       });
       __syncthreads();
       if (t == 0) {
-        int need = s_need, b = nb - 1;
-        for (; b > 0 && s_hist[b] < need; --b) need -= s_hist[b];
-        s_need = need;
-        s_prefix = prefix | ((uint32_t)b << sh);
-        s_mask = mask | ((uint32_t)(nb - 1) << sh);
+        int need = S.need, b = nb - 1;
+        for (; b > 0 && fh[b] < need; --b) need -= fh[b];
+        S.need = need;
+        S.prefix = prefix | ((uint32_t)b << sh);
+        S.mask = mask | ((uint32_t)(nb - 1) << sh);
       }
       __syncthreads();
     }
-    const uint32_t kth = s_prefix;          // key of the K-th largest value
-    const int need_eq = s_need;             // how many values equal to it are in the top K
+    const uint32_t kth = S.prefix;          // key of the K-th largest value
+    const int need_eq = S.need;             // how many values equal to it are in the top K
 
     // collection: values above the K-th, and the first need_eq equal to it
     const int per = (V + kSelectThreads - 1) / kSelectThreads;
@@ -195,7 +321,7 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
     int n_eq = 0;
     for (int v = b0; v < b1; ++v) n_eq += float_key(row[v]) == kth ? 1 : 0;
     int tot;
-    const int eq_before = block_exclusive_scan(n_eq, s_scan, &tot);
+    const int eq_before = block_exclusive_scan(n_eq, S.scan, &tot);
     for (int i = t; i < kMaxTopK; i += kSelectThreads) s_sort[i] = 0ull;
     __syncthreads();
     int eq_seen = eq_before;
@@ -207,7 +333,7 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
         ++eq_seen;
       }
       if (take) {
-        const int slot = atomicAdd(&s_found, 1);
+        const int slot = atomicAdd(&S.found, 1);
         if (slot < kMaxTopK) s_sort[slot] = pack_pair(k, v);
       }
     }
@@ -215,10 +341,170 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
     __syncthreads();
   }
   bitonic_sort_desc(s_sort, P);
+}
+
+// Appends the values of q (float4 u at float4 index i0 + u * kSelectThreads
+// of the row, present where bit u of `valid` is set) whose key is >= tau:
+// one shared atomic per value.  Returns whether this thread appended any;
+// sets *over when the list had no room.
+__device__ __forceinline__ bool append_block(SelShared& S, const float4 (&q)[kSelVec], uint32_t valid, int i0,
+                                             uint32_t tau, bool* over) {
+  float fmx = -INFINITY;
+  bool nan = false;
+#pragma unroll
+  for (int u = 0; u < kSelVec; ++u) {
+    fmx = fmaxf(fmx, fmaxf(fmaxf(q[u].x, q[u].y), fmaxf(q[u].z, q[u].w)));
+    nan |= (q[u].x != q[u].x) | (q[u].y != q[u].y) | (q[u].z != q[u].z) | (q[u].w != q[u].w);
+  }
+  // for a number x, key(x) >= tau exactly when x >= the float whose key is
+  // tau (a tau at or below the key of -inf bounds nothing); NaNs, whose keys
+  // lie beyond the infinities, are checked by key
+  if (!(tau <= 0x007fffffu || nan || fmx >= key_float(tau))) return false;
+  bool any = false;
+#pragma unroll
+  for (int u = 0; u < kSelVec; ++u) {
+    if (!((valid >> u) & 1u)) continue;
+    const float f[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t k = float_key(f[e]);
+      if (k >= tau) {
+        any = true;
+        const int slot = atomicAdd(&S.count, 1);
+        if (slot < kSelCap) S.list[slot] = pack_pair(k, 4 * (i0 + u * kSelectThreads) + e);
+        else *over = true;
+      }
+    }
+  }
+  return any;
+}
+
+// z: rows of `ldz` fp32 values (ldz a multiple of 4, rows 16-byte aligned),
+// the first V of each valid.  Writes K int32 indices and K fp32 logits per
+// row to idx_out / val_out (row r at out_row0 + r, K per row).
+__global__ void __launch_bounds__(kSelectThreads)
+topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int out_row0,
+                   int32_t* __restrict__ idx_out, float* __restrict__ val_out) {
+  __shared__ SelShared S;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const float* row = z + (size_t)blockIdx.x * ldz;
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  const int V4 = V >> 2;
+  const int nblocks = V4 > 0 ? (V4 + kSelBlock - 1) / kSelBlock : 1;
+
+  if (t == 0) {
+    S.count = 0;
+    S.over_flag = 0;
+  }
+  __syncthreads();
+
+  uint32_t tau = 0u;                      // keys below tau are never in the top K
+  bool fallback = false, mine = false, over = false;
+#pragma unroll 1
+  for (int b = 0; b < nblocks; ++b) {
+    // this block: float4 i0 + u * kSelectThreads, streamed (read once)
+    const int i0 = b * kSelBlock + t;
+    float4 q[kSelVec];
+    uint32_t valid = 0u;
+#pragma unroll
+    for (int u = 0; u < kSelVec; ++u) {
+      const int i = i0 + u * kSelectThreads;
+      if (i < V4) {
+        q[u] = __ldcs(r4 + i);
+        valid |= 1u << u;
+      } else {
+        q[u] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+    }
+    if (b == 0 && K <= 8 * 32) {
+      // a first threshold: in every warp, the ceil(K/8)-th largest of its
+      // lanes' maxima; the smallest of these 8 has at least K keys at or above it
+      uint32_t m = 0u;
+#pragma unroll
+      for (int u = 0; u < kSelVec; ++u)
+        if ((valid >> u) & 1u)
+          m = max(m, max(max(float_key(q[u].x), float_key(q[u].y)), max(float_key(q[u].z), float_key(q[u].w))));
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {        // descending bitonic sort of the warp's 32
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const uint32_t y = __shfl_xor_sync(0xffffffffu, m, stride);
+          const bool desc = (lane & size) == 0 || size == 32;
+          const bool lower = (lane & stride) == 0;
+          m = (lower == desc) ? max(m, y) : min(m, y);
+        }
+      }
+      const uint32_t kj = __shfl_sync(0xffffffffu, m, (K + 7) / 8 - 1);
+      if (lane == 0) S.wkey[w] = kj;
+      __syncthreads();
+      tau = S.wkey[0];
+#pragma unroll
+      for (int i = 1; i < kSelectThreads / 32; ++i) tau = min(tau, S.wkey[i]);
+    }
+    mine |= append_block(S, q, valid, i0, tau, &over);
+    if (b == nblocks - 1 && t == 0) {
+      // the scalar tail 4 V4 .. V-1 (fewer than 4 values)
+      for (int v = 4 * V4; v < V; ++v) {
+        const uint32_t k = float_key(row[v]);
+        if (k >= tau) {
+          mine = true;
+          const int slot = atomicAdd(&S.count, 1);
+          if (slot < kSelCap) S.list[slot] = pack_pair(k, v);
+          else over = true;
+        }
+      }
+    }
+    // the threads meet after the first block and then every kSelSegment
+    // blocks: one barrier when nothing was appended anywhere
+    if (b == 0 || b == nblocks - 1 || (b % kSelSegment) == 0) {
+      if (over) S.over_flag = 1;
+      if (!__syncthreads_or(mine || over)) continue;
+      mine = over = false;
+      const int n = S.count;
+      const bool any_over = S.over_flag != 0;
+      __syncthreads();
+      if (any_over) {                     // a candidate was lost: take the exact route
+        fallback = true;
+        break;
+      }
+      if (n > K && (b == 0 || n > kSelCap / 4)) {
+        // raise tau to the K-th largest key of the list and compact it
+        tau = kth_key(S, n, K);
+        const int m = compact_list(S, n, tau);
+        if (t == 0) S.count = m;
+        __syncthreads();
+        if (m > kSelCap / 4) {            // most of the list tied at tau
+          fallback = true;
+          break;
+        }
+      }
+    }
+  }
+
+  const unsigned long long* result = S.list;
+  if (!fallback && S.count < K) fallback = true;   // (not reached: tau keeps K keys at or above it)
+  if (!fallback) {
+    // cut the list to the keys at or above its K-th largest, and sort it
+    const int n = S.count;
+    int m = n;
+    if (n > K) {
+      const uint32_t kk = kth_key(S, n, K);
+      m = compact_list(S, n, kk);
+    }
+    int P = 1;
+    while (P < m) P <<= 1;
+    for (int i = m + t; i < P; i += kSelectThreads) S.list[i] = 0ull;   // below every real pair
+    __syncthreads();
+    bitonic_sort_desc(S.list, P);
+  } else {
+    __syncthreads();
+    select_two_pass(S, row, V, K);
+    result = fallback_sort(S);
+  }
 
   const size_t o = (size_t)(out_row0 + blockIdx.x) * K;
   for (int i = t; i < K; i += kSelectThreads) {
-    const unsigned long long e = s_sort[i];
+    const unsigned long long e = result[i];
     idx_out[o + i] = (int32_t)(0xffffffffu - (uint32_t)(e & 0xffffffffull));
     val_out[o + i] = key_float((uint32_t)(e >> 32));
   }

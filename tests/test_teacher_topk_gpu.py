@@ -108,3 +108,61 @@ def test_tied_rows(kd, V, K, n_pos):
     ridx, rval = oracle.teacher_topk(Ht, Wt, K)
     assert np.array_equal(idx, ridx)
     assert np.array_equal(val.astype(np.float64), rval)
+
+
+def _ordered_head(N, V, descending):
+    """A head whose logits are z[n, v] = v (or -v): H rows (4096, 64, 1, 0...)
+    and W rows (v // 4096, v // 64 % 64, v % 64, 0...) are exact in bf16, and
+    so are the integer logits in fp32."""
+    d = 16
+    Ht = torch.zeros(N, d)
+    Ht[:, 0], Ht[:, 1], Ht[:, 2] = 4096.0, 64.0, 1.0
+    if descending:
+        Ht = -Ht
+    v = torch.arange(V)
+    Wt = torch.zeros(V, d)
+    Wt[:, 0], Wt[:, 1], Wt[:, 2] = (v // 4096).float(), (v // 64 % 64).float(), (v % 64).float()
+    return Ht.to(torch.bfloat16), Wt.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("V,K,descending", [(70001, 100, False), (70001, 100, True), (40003, 512, False),
+                                            (9, 3, False)],
+                         ids=["ascending", "descending", "ascending_K512", "V9"])
+def test_ordered_rows(kd, V, K, descending):
+    """Rows in increasing column order make every block of the row the new
+    top K (the streaming select raises its threshold on each); decreasing
+    rows put it all in the first block."""
+    Ht, Wt = _ordered_head(5, V, descending)
+    idx, val = _gpu_topk(kd, Ht, Wt, K, chunk=4)
+    ridx, rval = oracle.teacher_topk(Ht, Wt, K)
+    assert np.array_equal(idx, ridx)
+    assert np.array_equal(val.astype(np.float64), rval)
+
+
+@pytest.mark.parametrize("N,d,V,K", [(40, 64, 70001, 100), (24, 32, 40000, 300)],
+                         ids=["V70001_K100", "V40000_K300"])
+def test_integer_logits_long_rows(kd, N, d, V, K):
+    """Rows many times the select's block length, with ties (integer logits)."""
+    g = torch.Generator().manual_seed(N * V + K)
+    Ht = torch.randint(-3, 4, (N, d), generator=g).to(torch.bfloat16)
+    Wt = torch.randint(-3, 4, (V, d), generator=g).to(torch.bfloat16)
+    idx, val = _gpu_topk(kd, Ht, Wt, K, chunk=16)
+    ridx, rval = oracle.teacher_topk(Ht, Wt, K)
+    assert np.array_equal(idx, ridx)
+    assert np.array_equal(val.astype(np.float64), rval)
+
+
+def test_infinite_logits(kd):
+    """+inf and -inf logits in a long row: +inf ranks above every finite
+    logit (and first in the cache), -inf below them."""
+    N, V, K = 4, 50001, 64
+    Ht, Wt = _ordered_head(N, V, descending=False)          # z[n, v] = v, exactly
+    W2 = Wt.clone().float()
+    W2[7, 0] = float("inf")                                  # z = +inf
+    W2[40000, 0] = float("-inf")                             # z = -inf
+    W2 = W2.to(torch.bfloat16)
+    idx, val = _gpu_topk(kd, Ht, W2, K, chunk=4)
+    ridx, rval = oracle.teacher_topk(Ht, W2, K)
+    assert np.isposinf(rval[:, 0]).all() and (ridx[:, 0] == 7).all()
+    assert np.array_equal(idx, ridx)
+    assert np.array_equal(val.astype(np.float64), rval)
