@@ -30,8 +30,8 @@
 // fit the sort buffer they are copied and sorted, otherwise a radix select
 // (12 + 8 more bits) finds the K-th largest key and a collection pass takes
 // every value above it and, of those equal to it, the ones with the lowest
-// column indices (threads own contiguous column ranges, so a scan of
-// per-thread counts orders them).
+// column indices (warps own contiguous column ranges and read them 32 columns
+// at a time; ballots and the counts of the warps before order the ties).
 #pragma once
 
 #include <cstdint>
@@ -66,23 +66,6 @@ __device__ __forceinline__ unsigned long long pack_pair(uint32_t k, int v) {
 
 __device__ __forceinline__ uint32_t pair_key(unsigned long long e) { return (uint32_t)(e >> 32); }
 
-// Block-wide exclusive scan of one int per thread (kSelectThreads threads).
-__device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int* total) {
-  const int t = threadIdx.x;
-  s_tmp[t] = v;
-  __syncthreads();
-  for (int off = 1; off < kSelectThreads; off <<= 1) {
-    const int x = t >= off ? s_tmp[t - off] : 0;
-    __syncthreads();
-    s_tmp[t] += x;
-    __syncthreads();
-  }
-  const int incl = s_tmp[t];
-  *total = s_tmp[kSelectThreads - 1];
-  __syncthreads();
-  return incl - v;
-}
-
 // Descending bitonic sort of s[0, P), P a power of two (all threads).
 __device__ __forceinline__ void bitonic_sort_desc(unsigned long long* s, int P) {
   for (int size = 2; size <= P; size <<= 1) {
@@ -108,8 +91,8 @@ __device__ __forceinline__ void bitonic_sort_desc(unsigned long long* s, int P) 
 struct SelShared {
   unsigned long long list[kSelCap];     // candidates (key, column)
   int fhist[4096];                      // the fallback's histogram
-  int hist[256];                        // radix histogram of the streaming route
-  int scan[kSelectThreads];
+  int hist[2][256];                     // radix histograms of the streaming route (alternating passes)
+  int scan[kSelectThreads / 32];          // the fallback's per-warp tie counts
   uint32_t wkey[kSelectThreads / 32];
   int count, found, need, ncand, over_flag;
   uint32_t prefix, mask;
@@ -119,16 +102,16 @@ static_assert(kCandCap <= kSelCap, "the fallback sorts in the candidate list");
 __device__ __forceinline__ unsigned long long* fallback_sort(SelShared& S) { return S.list; }
 __device__ __forceinline__ int* fallback_hist(SelShared& S) { return S.fhist; }
 
-// Warp 0: finds, in the 256-bin histogram, the highest bin b whose suffix sum
+// Warp 0: finds, in a 256-bin histogram, the highest bin b whose suffix sum
 // (bins b..255) reaches `need`, and writes S.prefix = prefix | b << sh and
 // S.need = the count still needed inside bin b.  Lane l owns bins 8l..8l+7.
 // With fewer than `need` values in all (not reached by the callers) bin 0.
-__device__ __forceinline__ void suffix_bin(SelShared& S, int need, uint32_t prefix, int sh) {
+__device__ __forceinline__ void suffix_bin(SelShared& S, const int* hist, int need, uint32_t prefix, int sh) {
   const int lane = threadIdx.x & 31;
   int c[8], own = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    c[i] = S.hist[8 * lane + i];
+    c[i] = hist[8 * lane + i];
     own += c[i];
   }
   int suf = own;                          // inclusive suffix sum over lanes
@@ -164,24 +147,27 @@ __device__ __forceinline__ void warp_hist_add(int* hist, bool pred, uint32_t bin
 }
 
 // Exact K-th largest key among list[0, n) (n >= K).  Radix select, 4 passes
-// of 8 bits.  All threads call it.
+// of 8 bits; pass p counts into hist[p & 1] while the other histogram is
+// cleared for the next pass, so a pass costs two barriers.  All threads call it.
 __device__ __forceinline__ uint32_t kth_key(SelShared& S, int n, int K) {
   const int t = threadIdx.x;
   const int lane = t & 31, w = t >> 5;
   uint32_t prefix = 0u, pmask = 0u;
   int need = K;
+  S.hist[0][t] = 0;
+  __syncthreads();
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int sh = 24 - 8 * pass;
-    S.hist[t] = 0;
-    __syncthreads();
+    int* hist = S.hist[pass & 1];
+    S.hist[(pass + 1) & 1][t] = 0;                                   // the next pass's histogram
     for (int base = 32 * w; base < n; base += kSelectThreads) {     // warp-uniform trip count
       const int i = base + lane;
       const uint32_t k = i < n ? pair_key(S.list[i]) : 0u;
-      warp_hist_add(S.hist, i < n && (k & pmask) == prefix, (k >> sh) & 255u);
+      warp_hist_add(hist, i < n && (k & pmask) == prefix, (k >> sh) & 255u);
     }
     __syncthreads();
-    if (t < 32) suffix_bin(S, need, prefix, sh);
+    if (t < 32) suffix_bin(S, hist, need, prefix, sh);
     __syncthreads();
     prefix = S.prefix;
     need = S.need;
@@ -192,29 +178,37 @@ __device__ __forceinline__ uint32_t kth_key(SelShared& S, int n, int K) {
 
 // Keeps the entries of list[0, n) whose key is >= tau (order not kept);
 // returns the new count.  Each thread reads its kSelCap / kSelectThreads
-// entries into registers before any is written.  All threads call it.
+// entries into registers, then the kept ones are appended again from 0 with
+// one shared atomic per warp.  All threads call it.
 __device__ __forceinline__ int compact_list(SelShared& S, int n, uint32_t tau) {
   constexpr int kPer = kSelCap / kSelectThreads;
-  const int t = threadIdx.x;
+  const int t = threadIdx.x, lane = t & 31;
   unsigned long long e[kPer];
   uint32_t keep = 0u;
-  int c = 0;
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int j = t * kPer + i;
     e[i] = j < n ? S.list[j] : 0ull;
-    if (j < n && pair_key(e[i]) >= tau) {
-      keep |= 1u << i;
-      ++c;
-    }
+    if (j < n && pair_key(e[i]) >= tau) keep |= 1u << i;
   }
-  int total;
-  int o = block_exclusive_scan(c, S.scan, &total);    // its barriers order every read before the writes
+  __syncthreads();                        // every entry read before any is overwritten
+  if (t == 0) S.count = 0;
+  __syncthreads();
+  const int cnt = __popc(keep);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  int base = 0;
+  if (lane == 31 && incl > 0) base = atomicAdd(&S.count, incl);
+  int o = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
 #pragma unroll
   for (int i = 0; i < kPer; ++i)
     if (keep & (1u << i)) S.list[o++] = e[i];
   __syncthreads();
-  return total;
+  return S.count;
 }
 
 // Calls f(v, value) for every column v < V of a row (16-byte aligned): four
@@ -315,27 +309,37 @@ __device__ __forceinline__ void select_two_pass(SelShared& S, const float* __res
     const int need_eq = S.need;             // how many values equal to it are in the top K
 
     // collection: values above the K-th, and the first need_eq equal to it
-    const int per = (V + kSelectThreads - 1) / kSelectThreads;
-    const int b0 = t * per;
-    const int b1 = (b0 + per < V) ? b0 + per : V;
-    int n_eq = 0;
-    for (int v = b0; v < b1; ++v) n_eq += float_key(row[v]) == kth ? 1 : 0;
-    int tot;
-    const int eq_before = block_exclusive_scan(n_eq, S.scan, &tot);
+    // in column order.  Warp w owns the contiguous columns [c0, c1) and reads
+    // them 32 at a time, lane l at column c0 + 32 i + l (coalesced); a ballot
+    // gives each lane its place among the warp's equal values, and a scan of
+    // the 8 warps' counts orders the warps.
+    const int lane = t & 31, w = t >> 5;
+    constexpr int kWarps = kSelectThreads / 32;
+    const int seg = ((V + kWarps - 1) / kWarps + 31) & ~31;
+    const int c0 = w * seg;
+    const int c1 = (c0 + seg < V) ? c0 + seg : V;
+    int n_eq = 0;                             // this warp's values equal to the K-th
+    for (int v0 = c0; v0 < c1; v0 += 32) {
+      const int v = v0 + lane;
+      n_eq += __popc(__ballot_sync(0xffffffffu, v < c1 && float_key(row[v < c1 ? v : c0]) == kth));
+    }
+    if (lane == 0) S.scan[w] = n_eq;
     for (int i = t; i < kMaxTopK; i += kSelectThreads) s_sort[i] = 0ull;
     __syncthreads();
-    int eq_seen = eq_before;
-    for (int v = b0; v < b1; ++v) {
-      const uint32_t k = float_key(row[v]);
-      bool take = k > kth;
-      if (k == kth) {
-        take = eq_seen < need_eq;
-        ++eq_seen;
-      }
+    int eq_seen = 0;                          // equal values in the warps before this one
+    for (int k = 0; k < w; ++k) eq_seen += S.scan[k];
+    for (int v0 = c0; v0 < c1; v0 += 32) {
+      const int v = v0 + lane;
+      const uint32_t k = v < c1 ? float_key(row[v]) : 0u;
+      const bool eq = v < c1 && k == kth;
+      const unsigned be = __ballot_sync(0xffffffffu, eq);
+      const int rank = eq_seen + __popc(be & ((1u << lane) - 1u));
+      const bool take = v < c1 && (k > kth || (eq && rank < need_eq));
       if (take) {
         const int slot = atomicAdd(&S.found, 1);
         if (slot < kMaxTopK) s_sort[slot] = pack_pair(k, v);
       }
+      eq_seen += __popc(be);
     }
     while (P < K) P <<= 1;
     __syncthreads();

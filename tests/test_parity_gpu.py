@@ -319,3 +319,42 @@ def test_calls_run_with_the_inputs_device_current(kd, monkeypatch):
     st, _ = kd.check(ws)
     assert st == 0
     assert len(seen) == 5 and all(d == g["H"].device for d in seen), seen
+
+
+@pytest.mark.parametrize("skip", [False, True], ids=["all_rows", "skip_masked_rows"])
+def test_fused_call_replays_in_a_cuda_graph(kd, skip):
+    """The fused call enqueues only stream work on the current stream
+    (memsets and kernel launches; skipped rows are counted on the device), so
+    a training loop can capture a step in a CUDA graph and replay it.  Each
+    replay must give the eager call's results bit for bit."""
+    N, d, V, K, chunk = 700, 512, 5000, 100, 256
+    g = _to_dev(workloads.make_inputs(_cfg(N, d, V, K, mask="drop5", seed=21)))
+    ws = kd.alloc_workspace(N, d, V, K, chunk, "cuda")
+    dH = torch.empty(N, d, dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty(V, d, dtype=torch.float32, device="cuda")
+
+    def step():
+        return kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0, chunk,
+                                   workspace=ws, dH=dH, dW=dW, skip_masked_rows=skip)
+
+    loss0, lse0, _, _ = step()
+    ref = (loss0.clone(), lse0.clone(), dH.clone(), dW.clone())
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()                                   # first calls on the capture stream happen before capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        loss, lse, _, _ = step()
+    for _ in range(2):
+        dH.fill_(1.0)
+        dW.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(loss, ref[0]) and torch.equal(lse, ref[1])
+        assert torch.equal(dH, ref[2]) and torch.equal(dW, ref[3])
+    st, _ = kd.check(ws)
+    assert st == 0
+    del graph
