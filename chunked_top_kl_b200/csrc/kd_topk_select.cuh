@@ -24,7 +24,8 @@
 //
 // For logits in no particular order the list stays small.  Rows where it
 // overflows (more candidates in one segment than the list holds: values
-// rising along the row, or heavy ties) are selected by the exact fallback
+// rising along the row, heavy ties, or K above 256, where the first block
+// has no threshold and fills the list) are selected by the exact fallback
 // below, which reads the row again: a histogram of the top 12 key bits
 // locates the bin of the K-th largest value; when the values in or above it
 // fit the sort buffer they are copied and sorted, otherwise a radix select
@@ -36,7 +37,6 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
-
 
 namespace kd {
 
@@ -92,7 +92,7 @@ struct SelShared {
   unsigned long long list[kSelCap];     // candidates (key, column)
   int fhist[4096];                      // the fallback's histogram
   int hist[2][256];                     // radix histograms of the streaming route (alternating passes)
-  int scan[kSelectThreads / 32];          // the fallback's per-warp tie counts
+  int scan[kSelectThreads / 32];        // the fallback's per-warp tie counts
   uint32_t wkey[kSelectThreads / 32];
   int count, found, need, ncand, over_flag;
   uint32_t prefix, mask;
