@@ -84,7 +84,7 @@ Layout make_layout(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk) {
   return L;
 }
 
-// The regions the forward pass alone uses, at the same offsets rules: status
+// The regions the forward pass alone uses, laid out as in make_layout: status
 // words, scalars, the fp64 block sums, the prepared teacher cache, the
 // per-split (m, s, g) partials and the forward's wave counters.  No dZ
 // chunk, no joint-launch counters, no row map or row buffers.  About
