@@ -364,16 +364,19 @@ def secondary_block(kd, dev, args, peaks):
     for n in cfg4.sweep:
         c = workloads.get_config(4, n)
         sweep.append(entry(c, measure_config(kd, c, dev, args.secondary_steps, 3)))
-    ns = [e["N"] for e in sweep]
-    gib = [e["peak_hbm_gib"] for e in sweep]
+    out[cfg4.name] = {"points": sweep,
+                      "peak_gib_fit": line_fit([e["N"] for e in sweep], [e["peak_hbm_gib"] for e in sweep])}
+    return out
+
+
+def line_fit(ns, gib):
+    """Least-squares line through peak GiB against tokens: its slope in bytes
+    per token, its intercept in GiB and the largest relative residual."""
     mn, mg = sum(ns) / len(ns), sum(gib) / len(gib)
     slope = sum((a - mn) * (b - mg) for a, b in zip(ns, gib)) / sum((a - mn) ** 2 for a in ns)
     icpt = mg - slope * mn
     resid = max(abs(b - (icpt + slope * a)) / b for a, b in zip(ns, gib))
-    out[cfg4.name] = {"points": sweep,
-                      "peak_gib_fit": {"slope_bytes_per_token": slope * 2**30, "intercept_gib": icpt,
-                                       "max_rel_residual": resid}}
-    return out
+    return {"slope_bytes_per_token": slope * 2**30, "intercept_gib": icpt, "max_rel_residual": resid}
 
 
 def run_cuda(args, cfg, world, rank, local):

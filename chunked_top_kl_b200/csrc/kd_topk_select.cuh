@@ -11,8 +11,8 @@
 // largest key among a subset of the values seen so far, so a value below it
 // is beaten by K others and can never be in the top K, while every value at
 // or above the final tau is on the list.  The first block of the row sets tau
-// to the smallest, over the warps, of each warp's ceil(K/8)-th largest lane
-// maximum (each warp then holds that many distinct values at or above it),
+// to the smallest, over the warps, of each warp's ceil(K/warps)-th largest
+// lane maximum (each warp then holds that many distinct values at or above it),
 // and then to the exact K-th largest key of the list; after every kSelSegment
 // blocks the threads meet, and when the list has grown past a quarter of its
 // capacity tau is raised to the exact K-th largest key of the list by a radix
@@ -24,8 +24,8 @@
 //
 // For logits in no particular order the list stays small.  Rows where it
 // overflows (more candidates in one segment than the list holds: values
-// rising along the row, heavy ties, or K above 256, where the first block
-// has no threshold and fills the list) are selected by the exact fallback
+// rising along the row, heavy ties, or K above 32 per warp, where the first
+// block has no threshold and fills the list) are selected by the exact fallback
 // below, which reads the row again: a histogram of the top 12 key bits
 // locates the bin of the K-th largest value; when the values in or above it
 // fit the sort buffer they are copied and sorted, otherwise a radix select
@@ -41,10 +41,11 @@
 namespace kd {
 
 constexpr int kSelectThreads = 256;
+constexpr int kSelWarps = kSelectThreads / 32;
 constexpr int kMaxTopK = 512;
 constexpr int kSelVec = 8;           // float4 loads per thread per block of the row
 constexpr int kSelBlock = kSelectThreads * kSelVec;   // float4s per block (8192 values)
-constexpr int kSelSegment = 4;       // blocks between two meetings of the threads
+constexpr int kSelSegment = 8;       // blocks between two meetings of the threads
 constexpr int kSelCap = 2048;        // candidate list (power of two, >= 2 kMaxTopK)
 constexpr int kCandCap = 2048;       // fallback sort buffer (power of two, >= kMaxTopK)
 
@@ -92,8 +93,8 @@ struct SelShared {
   unsigned long long list[kSelCap];     // candidates (key, column)
   int fhist[4096];                      // the fallback's histogram
   int hist[2][256];                     // radix histograms of the streaming route (alternating passes)
-  int scan[kSelectThreads / 32];        // the fallback's per-warp tie counts
-  uint32_t wkey[kSelectThreads / 32];
+  int scan[kSelWarps];                  // the fallback's per-warp tie counts
+  uint32_t wkey[kSelWarps];
   int count, found, need, ncand, over_flag;
   uint32_t prefix, mask;
 };
@@ -154,13 +155,13 @@ __device__ __forceinline__ uint32_t kth_key(SelShared& S, int n, int K) {
   const int lane = t & 31, w = t >> 5;
   uint32_t prefix = 0u, pmask = 0u;
   int need = K;
-  S.hist[0][t] = 0;
+  for (int i = t; i < 256; i += kSelectThreads) S.hist[0][i] = 0;
   __syncthreads();
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int sh = 24 - 8 * pass;
     int* hist = S.hist[pass & 1];
-    S.hist[(pass + 1) & 1][t] = 0;                                   // the next pass's histogram
+    for (int i = t; i < 256; i += kSelectThreads) S.hist[(pass + 1) & 1][i] = 0;  // next pass
     for (int base = 32 * w; base < n; base += kSelectThreads) {     // warp-uniform trip count
       const int i = base + lane;
       const uint32_t k = i < n ? pair_key(S.list[i]) : 0u;
@@ -314,8 +315,7 @@ __device__ __forceinline__ void select_two_pass(SelShared& S, const float* __res
     // gives each lane its place among the warp's equal values, and a scan of
     // the 8 warps' counts orders the warps.
     const int lane = t & 31, w = t >> 5;
-    constexpr int kWarps = kSelectThreads / 32;
-    const int seg = ((V + kWarps - 1) / kWarps + 31) & ~31;
+    const int seg = ((V + kSelWarps - 1) / kSelWarps + 31) & ~31;
     const int c0 = w * seg;
     const int c1 = (c0 + seg < V) ? c0 + seg : V;
     int n_eq = 0;                             // this warp's values equal to the K-th
@@ -420,9 +420,9 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
         q[u] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
       }
     }
-    if (b == 0 && K <= 8 * 32) {
-      // a first threshold: in every warp, the ceil(K/8)-th largest of its
-      // lanes' maxima; the smallest of these 8 has at least K keys at or above it
+    if (b == 0 && K <= kSelWarps * 32) {
+      // a first threshold: in every warp, the ceil(K/warps)-th largest of its
+      // lanes' maxima; the smallest of these has at least K keys at or above it
       uint32_t m = 0u;
 #pragma unroll
       for (int u = 0; u < kSelVec; ++u)
@@ -438,12 +438,12 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
           m = (lower == desc) ? max(m, y) : min(m, y);
         }
       }
-      const uint32_t kj = __shfl_sync(0xffffffffu, m, (K + 7) / 8 - 1);
+      const uint32_t kj = __shfl_sync(0xffffffffu, m, (K + kSelWarps - 1) / kSelWarps - 1);
       if (lane == 0) S.wkey[w] = kj;
       __syncthreads();
       tau = S.wkey[0];
 #pragma unroll
-      for (int i = 1; i < kSelectThreads / 32; ++i) tau = min(tau, S.wkey[i]);
+      for (int i = 1; i < kSelWarps; ++i) tau = min(tau, S.wkey[i]);
     }
     mine |= append_block(S, q, valid, i0, tau, &over);
     if (b == nblocks - 1 && t == 0) {

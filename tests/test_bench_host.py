@@ -91,3 +91,20 @@ def test_teacher_topk_mode_host_logic():
     out = _run_bench(["--op", "teacher-topk", "--impl", "reference", "--config", "0", "--steps", "1",
                       "--warmup", "3"])
     assert out.returncode != 0 and "teacher-topk" in out.stderr
+
+
+def test_peak_memory_line_fit():
+    """The secondary block's least-squares line through peak GiB against N:
+    exact on points on a line, and the largest relative residual it reports
+    is that of the point off the line."""
+    sys.path.insert(0, ROOT)
+    import bench
+    ns = [4096, 16384, 32768, 65536, 131072, 262144]
+    gib = [2.5 + n * 10000 / 2**30 for n in ns]
+    fit = bench.line_fit(ns, gib)
+    assert abs(fit["slope_bytes_per_token"] - 10000) < 1e-6
+    assert abs(fit["intercept_gib"] - 2.5) < 1e-9
+    assert fit["max_rel_residual"] < 1e-12
+    gib[2] *= 1.01                                     # one point 1 % high
+    fit = bench.line_fit(ns, gib)
+    assert 0.005 < fit["max_rel_residual"] < 0.011
