@@ -1,0 +1,112 @@
+"""GPU parity at the edges of the supported shapes, against the fp64 oracle
+(tolerances as everywhere: loss relative 1e-3, lse absolute 2e-3, dH and dW
+relative Frobenius 1e-2):
+
+* the largest teacher top-K (512) and a wide hidden size (4096);
+* a one-column vocabulary (V = K = 1: the teacher and the student agree
+  exactly, so the loss and both gradients are zero, the GPU's within
+  rounding; lse is the single logit);
+* skipping masked rows with one-token chunks, and with a single kept token.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from workloads.configs import Config
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-3
+LSE_ATOL = 2e-3
+GRAD_RFRO = 1e-2
+
+
+@pytest.fixture(scope="module")
+def kd():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from chunked_top_kl_b200 import build
+    build.build()
+    import chunked_top_kl_b200 as k
+    return k
+
+
+def _inputs(N, d, V, K, seed, mask="drop5"):
+    cfg = Config(f"edge_N{N}_d{d}_V{V}_K{K}", N, d, V, K, 1.0, 128, w_std=d ** -0.5,
+                 teacher="uniform", mask=mask, seed=seed)
+    return workloads.make_inputs(cfg)
+
+
+def _fused(kd, x, chunk, skip=False):
+    g = {k: v.cuda() for k, v in x.items()}
+    N, d = g["H"].shape
+    V, K = g["W"].shape[0], g["topk_idx"].shape[1]
+    ws = kd.alloc_workspace(N, d, V, K, chunk, "cuda")
+    loss, lse, dH, dW = kd.forward_backward(g["H"], g["W"], g["topk_idx"], g["topk_logit"], g["mask"], 1.0,
+                                            chunk, workspace=ws, skip_masked_rows=skip)
+    st, nbad = kd.check(ws)
+    assert st == 0 and nbad == 0, (kd.kd_status_string(st), nbad)
+    return {"loss": float(loss.item()), "lse": lse.double().cpu().numpy(),
+            "dH": dH.double().cpu().numpy(), "dW": dW.double().cpu().numpy()}
+
+
+def _rfro(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def _parity(got, x, what):
+    ref = oracle.kd_topk_kl(x["H"], x["W"], x["topk_idx"], x["topk_logit"], x["mask"], 1.0)
+    if ref["loss"] != 0.0:
+        assert abs(got["loss"] - ref["loss"]) <= LOSS_RTOL * abs(ref["loss"]), (what, got["loss"], ref["loss"])
+    else:
+        assert abs(got["loss"]) <= 1e-6, (what, got["loss"])
+    assert np.max(np.abs(got["lse"] - ref["lse"])) <= LSE_ATOL, what
+    for k in ("dH", "dW"):
+        assert _rfro(got[k], ref[k]) <= GRAD_RFRO, (what, k, _rfro(got[k], ref[k]))
+    return ref
+
+
+@pytest.mark.parametrize("N,d,V,K,chunk", [(200, 64, 3000, 512, 64), (130, 4096, 1000, 8, 128)],
+                         ids=["K512", "d4096"])
+def test_largest_K_and_wide_hidden(kd, N, d, V, K, chunk):
+    x = _inputs(N, d, V, K, seed=N + K)
+    _parity(_fused(kd, x, chunk), x, f"N{N}_d{d}_V{V}_K{K}")
+
+
+def test_one_column_vocabulary(kd):
+    x = _inputs(50, 64, 1, 1, seed=3, mask="ones")
+    got = _fused(kd, x, 16)
+    ref = _parity(got, x, "V1")             # the GPU values within rounding of exact zeros
+    assert ref["loss"] == 0.0 and np.all(ref["dH"] == 0.0) and np.all(ref["dW"] == 0.0)
+    z = x["H"].double().numpy() @ x["W"].double().numpy().T
+    assert np.max(np.abs(got["lse"] - z[:, 0])) <= LSE_ATOL
+
+
+def test_skip_rows_with_one_token_chunks(kd):
+    x = _inputs(40, 64, 500, 8, seed=9, mask="ones")
+    g = torch.Generator().manual_seed(9)
+    x["mask"] = (torch.rand(40, generator=g) >= 0.3).float()
+    a = _fused(kd, x, 1, skip=False)
+    b = _fused(kd, x, 1, skip=True)
+    assert a["loss"] == b["loss"] and np.array_equal(a["lse"], b["lse"]) and np.array_equal(a["dH"], b["dH"])
+    assert _rfro(b["dW"], a["dW"]) <= 1e-5
+    _parity(b, x, "chunk=1 skip")
+
+
+def test_skip_rows_single_kept_token(kd):
+    x = _inputs(300, 72, 700, 6, seed=10, mask="ones")
+    x["mask"] = torch.zeros(300)
+    x["mask"][299] = 1.0
+    got = _fused(kd, x, 128, skip=True)
+    ref = _parity(got, x, "single kept token")
+    assert np.all(got["dH"][:299] == 0.0)
+    assert math.isclose(got["loss"], ref["term"][299], rel_tol=LOSS_RTOL)
+

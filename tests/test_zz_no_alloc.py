@@ -9,7 +9,7 @@ through the C ABI twice in a row on different inputs, at a GPT-OSS-shaped
 head (d = 2880, V = 201088) with the largest token count its scratch holds
 (checked against the fp64 oracle on sampled tokens too), and with a bad
 teacher index, which it reports as NaN (its caller has no workspace to read
-the status words from).  This file sorts last so that a run stopping at the
+the status words from), and on an empty batch.  This file sorts last so that a run stopping at the
 first failure has already run every other test.
 """
 
@@ -124,3 +124,19 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(kd):
                                        N, d, V, K, 1.0, loss.data_ptr(), lse.data_ptr(),
                                        torch.cuda.current_stream().cuda_stream)
     assert st == _abi.KD_ERR_WORKSPACE
+
+
+def test_noalloc_forward_on_an_empty_batch(kd):
+    """N = 0: nothing to read, the loss is written as 0 (an empty mask sum)."""
+    W = torch.randn(100, 64, device="cuda").to(torch.bfloat16)
+    H = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(0, 4, dtype=torch.int32, device="cuda")
+    lg = torch.empty(0, 4, dtype=torch.float32, device="cuda")
+    loss = torch.full((), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.empty(0, dtype=torch.float32, device="cuda")
+    st = kd.kd_topk_kl_forward_noalloc(H.data_ptr() or 256, W.data_ptr(), idx.data_ptr() or 256,
+                                       lg.data_ptr() or 256, 0, 0, 64, 100, 4, 1.0, loss.data_ptr(),
+                                       lse.data_ptr() or 256, torch.cuda.current_stream().cuda_stream)
+    assert st == 0, kd.kd_status_string(st)
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0
