@@ -836,6 +836,63 @@ struct EpiDw {
   }
 };
 
+// Teacher logits, per chunk: the fp32 tile stored like EpiDw's first chunk
+// (columns past V clipped by the tensor map), and per token row and tile the
+// order key (float_key) of the row's largest logit in the tile.  The top-K
+// selection takes its first threshold from these maxima and reads only the
+// tiles that can hold a top-K logit.
+struct EpiZ32 {
+  static constexpr bool kStaging = true;
+  struct Params {
+    uint32_t* tmax;       // [rows][ld] keys
+    int ld;               // tiles per row, ceil(V / BN)
+    int rows;             // token rows of the chunk
+    int V;
+  };
+  __device__ __forceinline__ void begin_unit(const Params&, int, int, int, const EpiCtx&) {}
+  __device__ __forceinline__ void end_unit(const Params&, int, int) {}
+
+  __device__ __forceinline__ void tile(const Params& P, const CUtensorMap* out, int grow, int n,
+                                       uint32_t taddr, EpiCtx& cx) {
+    float fmx = -INFINITY;                // max of the logits, NaN if any is NaN
+#pragma unroll 1
+    for (int j = 0; j < BN / 32; ++j) {
+      const int c0 = n * BN + j * 32;
+      float v[32];
+      __syncwarp();
+      tmem_ld_32x32b_x32(taddr + j * 32, v);
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+      if (c0 + 32 <= P.V) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) fmx = fmax_nan(fmx, v[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c0 + i < P.V) fmx = fmax_nan(fmx, v[i]);
+      }
+      stage_store(cx, out, c0, cx.row_base, w, false);
+    }
+    uint32_t key = float_key(fmx);
+    if (__any_sync(0xffffffffu, fmx != fmx)) {   // NaNs order by key: take the maximum key itself
+      uint32_t km = 0u;
+#pragma unroll 1
+      for (int j = 0; j < BN / 32; ++j) {
+        const int c0 = n * BN + j * 32;
+        float v[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(taddr + j * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c0 + i < P.V) km = max(km, float_key(v[i]));
+      }
+      key = km;
+    }
+    if (grow < P.rows) P.tmax[(size_t)grow * P.ld + n] = key;
+  }
+};
+
 // Placeholder epilogue of an absent second problem.
 struct EpiNone {
   static constexpr bool kStaging = false;

@@ -377,6 +377,13 @@ __device__ __forceinline__ bool epilogue_bar_and(uint32_t count, bool pred) {
   return out != 0;
 }
 
+// max(a, b), NaN when either is NaN (PTX max.NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint16_t ld_shared_u16(uint32_t addr) {
   uint16_t v;
   asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");

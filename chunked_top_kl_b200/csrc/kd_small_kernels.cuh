@@ -22,6 +22,19 @@ struct Status {
   unsigned int pad[14];
 };
 
+// Order-preserving map of a float onto uint32 (larger float, larger key;
+// NaNs with the sign bit clear above +inf, with it set below -inf).  The
+// teacher top-K selection compares logits by these keys.
+__device__ __forceinline__ uint32_t float_key(float v) {
+  if (v == 0.f) v = 0.f;                // -0 and +0 are one value
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -282,7 +282,7 @@ using ProbFwd = Prob<EpiFwd, false, false, kL2EvictLast, kL2Normal>;  // A = H (
 using ProbDz = Prob<EpiDz, false, false, kL2EvictLast, kL2Normal>;    // A = H chunk, B = W
 using ProbDh = Prob<EpiDh, false, true>;      // A = dZ (K-major over V), B = W (MN-major over d)
 using ProbDw = Prob<EpiDw, true, true, kL2Normal, kL2EvictLast>;      // A = dZ^T (MN-major over V), B = H chunk
-using ProbZ32 = Prob<EpiDw, false, false, kL2EvictLast, kL2Normal>;   // teacher logits, fp32 store: A = Ht, B = Wt
+using ProbZ32 = Prob<EpiZ32, false, false, kL2EvictLast, kL2Normal>;  // teacher logits, fp32 store: A = Ht, B = Wt
 
 // The loss as one call computes it: the teacher logits and their type, T,
 // and the factors of the student-temperature variant (zs on the student
@@ -731,25 +731,29 @@ int kd_topk_kl_check(const void* workspace, void* stream, int64_t* bad_index_cou
 // logits of the teacher head and their indices (blog post, "Two systems
 // changes", offline distillation paragraph).  Per chunk of tokens, the
 // teacher logits z = Ht Wt^T are computed by the same tcgen05 GEMM as the
-// loss (fp32 tiles stored through TMA into a chunk buffer) and each row's
-// top K are selected exactly (topk_select_kernel).
+// loss (fp32 tiles stored through TMA into a chunk buffer, with the largest
+// logit of every row's 256-column tile kept beside them) and each row's top
+// K are selected exactly (topk_select_kernel), reading only the tiles whose
+// maximum can be among them.
 
 namespace {
 
 // Status words first (as in the loss workspace, so kd_topk_kl_check reads
-// them), then one chunk of fp32 logits.
+// them), then one chunk of fp32 logits and the keys of their tile maxima.
 struct TopkLayout {
-  int64_t C = 0, ldz = 0;
-  size_t off_status = 0, off_z = 0, total = 0;
+  int64_t C = 0, ldz = 0, tmld = 0;
+  size_t off_status = 0, off_z = 0, off_tmax = 0, total = 0;
 };
 
 TopkLayout make_topk_layout(int64_t N, int64_t V, int64_t chunk) {
   TopkLayout L;
   L.C = N > 0 ? (chunk < N ? chunk : N) : 1;
   L.ldz = round_up(V, 4);
+  L.tmld = ceil_div(V, BN);
   L.off_status = 0;
   L.off_z = align256(sizeof(Status));
-  L.total = L.off_z + align256(sizeof(float) * (size_t)L.C * L.ldz);
+  L.off_tmax = L.off_z + align256(sizeof(float) * (size_t)L.C * L.ldz);
+  L.total = L.off_tmax + align256(sizeof(uint32_t) * (size_t)L.C * L.tmld);
   return L;
 }
 
@@ -788,6 +792,7 @@ int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_
   if (cudaGetDevice(&dev) != cudaSuccess) return KD_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KD_ERR_UNSUPPORTED;
   float* zbuf = at<float>(workspace, L.off_z);
+  uint32_t* tmax = at<uint32_t>(workspace, L.off_tmax);
 
   CUtensorMap tmH, tmW;
   if (!make_map(&tmH, Ht, d, N, d, BK, BM) || !make_map(&tmW, Wt, d, V, d, BK, GeoP::B_ROWS)) return KD_ERR_CUDA;
@@ -801,12 +806,15 @@ int kd_teacher_topk(const void* Ht, const void* Wt, int64_t N, int64_t d, int64_
     a.raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(V, BN), true);
     a.num_kb = (int)ceil_div(d, BK);
     a.a_row0 = (int)c0;
-    EpiDw::Params e{};
-    e.accumulate = 0;
+    EpiZ32::Params e{};
+    e.tmax = tmax;
+    e.ld = (int)L.tmld;
+    e.rows = (int)Cc;
+    e.V = (int)V;
     if (launch_one<ProbZ32>(3, dev, grid_for(a.raster, groups), tmH, tmW, tmZ, a, status, e, s) != cudaSuccess)
       return KD_ERR_CUDA;
     topk_select_kernel<<<(unsigned)Cc, kSelectThreads, 0, s>>>(zbuf, L.ldz, (int)V, (int)K, (int)c0, topk_idx,
-                                                               topk_logit);
+                                                               topk_logit, tmax, (int)L.tmld);
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
   return KD_OK;

@@ -3,40 +3,53 @@
 // equal values in increasing column order (the order in which an offline
 // cache lists a position's top-K teacher logits).
 //
-// One CTA per row, values mapped to order-preserving 32-bit keys, and one
-// read of the row.  The threads stream the row with 16-byte loads (kSelVec of
-// them in flight per thread, consecutive threads on consecutive addresses),
-// and a value becomes a candidate, appended to a shared-memory list, when
-// its key is at least the current threshold tau.  tau is always the K-th
-// largest key among a subset of the values seen so far, so a value below it
-// is beaten by K others and can never be in the top K, while every value at
-// or above the final tau is on the list.  The first block of the row sets tau
-// to the smallest, over the warps, of each warp's ceil(K/warps)-th largest
-// lane maximum (each warp then holds that many distinct values at or above it),
-// and then to the exact K-th largest key of the list; after every kSelSegment
-// blocks the threads meet, and when the list has grown past a quarter of its
-// capacity tau is raised to the exact K-th largest key of the list by a radix
-// select over shared memory and the list is compacted.  A thread first
-// compares the maximum of its values with tau in floats and only then looks
-// at single values, so after the first blocks a value costs a load and a max.
-// At the end the list is cut to the keys at or above its K-th largest and
-// sorted by (key desc, column asc).
+// One CTA per row, values mapped to order-preserving 32-bit keys.  The
+// threads stream 16-byte loads (kSelVec of them in flight per thread) and a
+// value becomes a candidate, appended to a shared-memory list, when its key is
+// at least the current threshold tau.  tau is always the K-th largest key
+// among a subset of the row's values, so a value below it is beaten by K
+// others and can never be in the top K, while every value at or above the
+// final tau is on the list.
+//
+// Which values are streamed.  The logits GEMM also writes, per row and
+// 256-column tile, the key of the tile's largest value (EpiZ32).  With at
+// least K tiles, tau starts at the K-th largest of these maxima (a radix
+// select over shared memory): the K tiles with the largest maxima hold K
+// values at or above it, so every value at or above the row's K-th largest
+// is at or above tau and lies in a tile whose maximum is too, and only those
+// tiles are read: about K of the row's tiles for logits in no particular
+// order (at V = 201,088 and K = 100, 1/8 of the row).  Without the maxima, or
+// with fewer than K tiles, the whole row is streamed (consecutive threads on
+// consecutive addresses), and the first block sets tau to the smallest, over
+// the warps, of each warp's ceil(K/warps)-th largest lane maximum (each warp
+// then holds that many distinct values at or above it).
+//
+// Either way tau is then raised to the exact K-th largest key of the list
+// after the first block, and whenever the threads meet (every kSelSegment
+// blocks) with the list past a quarter of its capacity, and the list is
+// compacted.  A thread first compares the maximum of its values with tau in
+// floats and only then looks at single values, so after the first blocks a
+// value costs a load and a max.  At the end the list is cut to the keys at or
+// above its K-th largest and sorted by (key desc, column asc).
 //
 // For logits in no particular order the list stays small.  Rows where it
 // overflows (more candidates in one segment than the list holds: values
-// rising along the row, heavy ties, or K above 32 per warp, where the first
-// block has no threshold and fills the list) are selected by the exact fallback
-// below, which reads the row again: a histogram of the top 12 key bits
-// locates the bin of the K-th largest value; when the values in or above it
-// fit the sort buffer they are copied and sorted, otherwise a radix select
-// (12 + 8 more bits) finds the K-th largest key and a collection pass takes
-// every value above it and, of those equal to it, the ones with the lowest
-// column indices (warps own contiguous column ranges and read them 32 columns
-// at a time; ballots and the counts of the warps before order the ties).
+// rising along the row, heavy ties, or, streaming the whole row, K above 32
+// per warp, where the first block has no threshold and fills the list) are
+// selected by the exact fallback below, which reads the whole row again: a
+// histogram of the top 12 key bits locates the bin of the K-th largest value;
+// when the values in or above it fit the sort buffer they are copied and
+// sorted, otherwise a radix select (12 + 8 more bits) finds the K-th largest
+// key and a collection pass takes every value above it and, of those equal
+// to it, the ones with the lowest column indices (warps own contiguous column
+// ranges and read them 32 columns at a time; ballots and the counts of the
+// warps before order the ties).
 #pragma once
 
 #include <cstdint>
 #include <cuda_runtime.h>
+
+#include "kd_small_kernels.cuh"
 
 namespace kd {
 
@@ -46,19 +59,10 @@ constexpr int kMaxTopK = 512;
 constexpr int kSelVec = 8;           // float4 loads per thread per block of the row
 constexpr int kSelBlock = kSelectThreads * kSelVec;   // float4s per block (8192 values)
 constexpr int kSelSegment = 8;       // blocks between two meetings of the threads
+constexpr int kSelTile = 256;        // columns per tile maximum (the logits GEMM's tile width)
+constexpr int kSelTilesPerBlock = kSelBlock / (kSelTile / 4);   // tiles per block of the tile route
 constexpr int kSelCap = 2048;        // candidate list (power of two, >= 2 kMaxTopK)
 constexpr int kCandCap = 2048;       // fallback sort buffer (power of two, >= kMaxTopK)
-
-// Order-preserving map of a float onto uint32 (larger float, larger key).
-__device__ __forceinline__ uint32_t float_key(float v) {
-  if (v == 0.f) v = 0.f;                // -0 and +0 are one value
-  const uint32_t u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float key_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
 
 // A (key, column) pair as one sortable word: larger key first, then lower column.
 __device__ __forceinline__ unsigned long long pack_pair(uint32_t k, int v) {
@@ -95,7 +99,7 @@ struct SelShared {
   int hist[2][256];                     // radix histograms of the streaming route (alternating passes)
   int scan[kSelWarps];                  // the fallback's per-warp tie counts
   uint32_t wkey[kSelWarps];
-  int count, found, need, ncand, over_flag;
+  int count, found, need, ncand, over_flag, ntsel;
   uint32_t prefix, mask;
 };
 static_assert(kCandCap <= kSelCap, "the fallback sorts in the candidate list");
@@ -347,12 +351,13 @@ __device__ __forceinline__ void select_two_pass(SelShared& S, const float* __res
   bitonic_sort_desc(s_sort, P);
 }
 
-// Appends the values of q (float4 u at float4 index i0 + u * kSelectThreads
-// of the row, present where bit u of `valid` is set) whose key is >= tau:
-// one shared atomic per value.  Returns whether this thread appended any;
-// sets *over when the list had no room.
-__device__ __forceinline__ bool append_block(SelShared& S, const float4 (&q)[kSelVec], uint32_t valid, int i0,
-                                             uint32_t tau, bool* over) {
+// Appends to the list every value of q (a block of the row: value e of
+// q[u] is column 4 col4(u) + e, present where bit u of `valid` is set) whose
+// key is >= tau: one shared atomic per value.  Returns whether this thread
+// appended any; sets *over when the list had no room.
+template <class Col4>
+__device__ __forceinline__ bool append_block(SelShared& S, const float4 (&q)[kSelVec], uint32_t valid,
+                                             const Col4& col4, uint32_t tau, bool* over) {
   float fmx = -INFINITY;
   bool nan = false;
 #pragma unroll
@@ -375,7 +380,7 @@ __device__ __forceinline__ bool append_block(SelShared& S, const float4 (&q)[kSe
       if (k >= tau) {
         any = true;
         const int slot = atomicAdd(&S.count, 1);
-        if (slot < kSelCap) S.list[slot] = pack_pair(k, 4 * (i0 + u * kSelectThreads) + e);
+        if (slot < kSelCap) S.list[slot] = pack_pair(k, 4 * col4(u) + e);
         else *over = true;
       }
     }
@@ -384,43 +389,82 @@ __device__ __forceinline__ bool append_block(SelShared& S, const float4 (&q)[kSe
 }
 
 // z: rows of `ldz` fp32 values (ldz a multiple of 4, rows 16-byte aligned),
-// the first V of each valid.  Writes K int32 indices and K fp32 logits per
-// row to idx_out / val_out (row r at out_row0 + r, K per row).
+// the first V of each valid.  tmax (or null): per row, `tmld` order keys, the
+// largest of each 256-column tile of the row (EpiZ32).  Writes K int32
+// indices and K fp32 logits per row to idx_out / val_out (row r at
+// out_row0 + r, K per row).
 __global__ void __launch_bounds__(kSelectThreads)
 topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int out_row0,
-                   int32_t* __restrict__ idx_out, float* __restrict__ val_out) {
+                   int32_t* __restrict__ idx_out, float* __restrict__ val_out,
+                   const uint32_t* __restrict__ tmax, int tmld) {
   __shared__ SelShared S;
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
   const float* row = z + (size_t)blockIdx.x * ldz;
   const float4* r4 = reinterpret_cast<const float4*>(row);
   const int V4 = V >> 2;
-  const int nblocks = V4 > 0 ? (V4 + kSelBlock - 1) / kSelBlock : 1;
+  const int ntiles = (V + kSelTile - 1) / kSelTile;
 
   if (t == 0) {
     S.count = 0;
     S.over_flag = 0;
+    S.ntsel = 0;
   }
   __syncthreads();
 
   uint32_t tau = 0u;                      // keys below tau are never in the top K
+  // The tile route: tau = the K-th largest tile maximum.  The K tiles with
+  // the largest maxima hold K values at or above it, so every value at or
+  // above the row's K-th largest is at or above tau, and sits in a tile whose
+  // maximum is too: only those tiles are read.
+  const bool by_tile = tmax != nullptr && ntiles >= K && ntiles <= kSelCap;
+  int* tsel = S.fhist;                    // the selected tiles (the fallback's histogram is free)
+  int nsel = 0;
+  if (by_tile) {
+    const uint32_t* trow = tmax + (size_t)blockIdx.x * tmld;
+    for (int i = t; i < ntiles; i += kSelectThreads) S.list[i] = pack_pair(trow[i], i);
+    __syncthreads();
+    tau = kth_key(S, ntiles, K);
+    for (int i = t; i < ntiles; i += kSelectThreads)
+      if (pair_key(S.list[i]) >= tau) tsel[atomicAdd(&S.ntsel, 1)] = i;
+    __syncthreads();
+    nsel = S.ntsel;
+  }
+  const int nblocks = by_tile ? (nsel + kSelTilesPerBlock - 1) / kSelTilesPerBlock
+                              : (V4 > 0 ? (V4 + kSelBlock - 1) / kSelBlock : 1);
+
   bool fallback = false, mine = false, over = false;
 #pragma unroll 1
   for (int b = 0; b < nblocks; ++b) {
-    // this block: float4 i0 + u * kSelectThreads, streamed (read once)
+    // float4 u of this thread: the row's float4 col4(u), streamed (read once)
+    // full row: b kSelBlock + t + u kSelectThreads; by tile: float4 t mod 64
+    // of the block's tile u (kSelectThreads / 64) + t / 64
     const int i0 = b * kSelBlock + t;
+    const int s0 = b * kSelTilesPerBlock + (t >> 6);
+    auto col4 = [&](int u) -> int {
+      return by_tile ? tsel[s0 + u * (kSelectThreads / 64)] * (kSelTile / 4) + (t & 63) : i0 + u * kSelectThreads;
+    };
     float4 q[kSelVec];
     uint32_t valid = 0u;
 #pragma unroll
     for (int u = 0; u < kSelVec; ++u) {
-      const int i = i0 + u * kSelectThreads;
-      if (i < V4) {
+      bool ok;
+      int i;
+      if (by_tile) {
+        ok = s0 + u * (kSelectThreads / 64) < nsel;
+        i = ok ? col4(u) : 0;
+        ok = ok && i < V4;
+      } else {
+        i = i0 + u * kSelectThreads;
+        ok = i < V4;
+      }
+      if (ok) {
         q[u] = __ldcs(r4 + i);
         valid |= 1u << u;
       } else {
         q[u] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
       }
     }
-    if (b == 0 && K <= kSelWarps * 32) {
+    if (!by_tile && b == 0 && K <= kSelWarps * 32) {
       // a first threshold: in every warp, the ceil(K/warps)-th largest of its
       // lanes' maxima; the smallest of these has at least K keys at or above it
       uint32_t m = 0u;
@@ -445,9 +489,10 @@ topk_select_kernel(const float* __restrict__ z, int64_t ldz, int V, int K, int o
 #pragma unroll
       for (int i = 1; i < kSelWarps; ++i) tau = min(tau, S.wkey[i]);
     }
-    mine |= append_block(S, q, valid, i0, tau, &over);
+    mine |= append_block(S, q, valid, col4, tau, &over);
     if (b == nblocks - 1 && t == 0) {
-      // the scalar tail 4 V4 .. V-1 (fewer than 4 values)
+      // the scalar tail 4 V4 .. V-1 (fewer than 4 values; appended whenever at
+      // or above tau, whichever route, which keeps every candidate)
       for (int v = 4 * V4; v < V; ++v) {
         const uint32_t k = float_key(row[v]);
         if (k >= tau) {

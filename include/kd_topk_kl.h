@@ -264,8 +264,10 @@ int kd_topk_kl_forward_backward_ex(const void* H, const void* W,
  * column indices, largest first, equal logits in increasing column order:
  * topk_idx int32 [N][K], topk_logit fp32 [N][K] (device, caller-owned).
  * Tokens are processed `chunk` at a time: the logits of one chunk are stored
- * in the workspace (chunk x round_up(V, 4) fp32) and each row's top K is
- * selected exactly.  Supported: 1 <= K <= min(V, 512), d % 8 == 0; Ht and Wt
+ * in the workspace (chunk x round_up(V, 4) fp32, and per row the largest
+ * logit of each 256-column tile) and each row's top K is selected exactly,
+ * reading only the tiles whose maximum reaches the K-th largest tile
+ * maximum when the row has at least K tiles.  Supported: 1 <= K <= min(V, 512), d % 8 == 0; Ht and Wt
  * 16-byte aligned, the workspace 256-byte aligned.  kd_topk_kl_check on this
  * workspace reports a pipeline timeout. */
 size_t kd_teacher_topk_workspace_size(int64_t N, int64_t d, int64_t V, int64_t K, int64_t chunk);

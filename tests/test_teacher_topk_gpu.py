@@ -4,6 +4,10 @@ fp64 oracle ``oracle.teacher_topk``.
 * Integer-valued H and W (exact in bf16, and every logit an integer well
   inside fp32's exact range): the GPU logits equal the oracle's exactly, so
   indices and logits must match bit for bit, ties (many of them) included.
+  With at least K tiles of 256 columns the selection reads only the tiles
+  whose maximum reaches the K-th largest tile maximum, otherwise the whole
+  row; the cases cover both, K equal to the number of tiles (every tile
+  read) and one past it.
 * Gaussian H and W at a few shapes (ragged N, V and chunk): the logits match
   within fp32 accumulation error, and the index sets match except where the
   oracle's K-th and (K+1)-th logits are closer than that error.
@@ -38,8 +42,10 @@ def _gpu_topk(kd, Ht, Wt, K, chunk):
     return idx.cpu().numpy(), val.cpu().numpy()
 
 
-@pytest.mark.parametrize("N,d,V,K,chunk", [(300, 64, 5000, 100, 128), (77, 16, 700, 7, 32), (40, 8, 300, 300, 64)],
-                         ids=["N300_V5000_K100", "N77_V700_K7", "K_equals_V"])
+@pytest.mark.parametrize("N,d,V,K,chunk", [(300, 64, 5000, 100, 128), (77, 16, 700, 7, 32), (40, 8, 300, 300, 64),
+                                           (128, 64, 4096, 16, 64), (128, 64, 4096, 17, 64), (100, 32, 3001, 5, 64)],
+                         ids=["N300_V5000_K100", "N77_V700_K7", "K_equals_V",
+                              "K_equals_tiles", "K_one_past_tiles", "V3001_K5_tiles"])
 def test_integer_logits_exact(kd, N, d, V, K, chunk):
     g = torch.Generator().manual_seed(N + V)
     Ht = torch.randint(-3, 4, (N, d), generator=g).to(torch.bfloat16)
