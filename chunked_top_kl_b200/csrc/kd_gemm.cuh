@@ -55,6 +55,7 @@ struct Geo {
   static constexpr int STAGING_BYTES = STAGING ? 2 * BM * 128 : 0;  // two 128-row x 128-byte buffers
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;  // per stage, whole tile
+  static constexpr uint32_t TX_B_BYTES = (PAIR ? 2 : 1) * B_BYTES;    // per stage holding only B (wide units)
 };
 
 // One GEMM as the kernel sees it: its tile schedule, K blocks per tile, and
@@ -68,7 +69,15 @@ struct ProbArgs {
                         // unit, 3: band x column range units) or its K (2)
   int dyn_bands_fastest;
   int dyn_zero_fill;    // role 2 with no live rows: still write the (zero) output tiles
+  int wide_cols;        // > 0: wide units (Prob WIDE): its 256-column tiles; the raster counts pairs of them
 };
+
+// K blocks of MMA work per unit of a problem, the joint schedule's cost: a
+// wide unit's K block runs two MMA blocks (one per column tile).  A problem
+// declared WIDE runs wide units when the launch sets wide_cols.
+KD_HD int64_t unit_cost(const ProbArgs& pa) {
+  return (int64_t)pa.raster.tiles_per_split * pa.num_kb * (pa.wide_cols > 0 ? 2 : 1);
+}
 
 // A launch over rows whose number is known only on the device (a chunk of the
 // compacted token list): the host plans `chunk` rows; every thread of the
@@ -124,24 +133,29 @@ __device__ __forceinline__ void apply_live_rows(GemmArgs& a, int rows, int ngrou
     }
   }
   if constexpr (HAS_P1)
-    a.joint = joint_plan(a.prob[0].raster.num_units, (int64_t)a.prob[0].raster.tiles_per_split * a.prob[0].num_kb,
-                         a.prob[1].raster.num_units, (int64_t)a.prob[1].raster.tiles_per_split * a.prob[1].num_kb,
-                         ngroups);
+    a.joint = joint_plan(a.prob[0].raster.num_units, unit_cost(a.prob[0]), a.prob[1].raster.num_units,
+                         unit_cost(a.prob[1]), ngroups);
 }
 
 // Compile-time description of a problem: its epilogue, operand majorness,
-// and the L2 eviction priority of each operand's loads (L2Hint).
-template <class EpiT, bool AMN, bool BMN, int AH = kL2Normal, int BH = kL2Normal>
+// the L2 eviction priority of each operand's loads (L2Hint), and whether its
+// units are wide.  A wide unit computes two neighbouring 256-column tiles of
+// one band (column tiles 2n and 2n + 1 for raster column n) into the two
+// accumulators at once, so each K block's A tile is loaded once for both:
+// three quarters of the operand bytes per MMA block of a one-tile unit.  The
+// epilogue of a wide unit cannot overlap the next unit's MMAs, so wide units
+// suit problems whose tiles run many K blocks.
+template <class EpiT, bool AMN, bool BMN, int AH = kL2Normal, int BH = kL2Normal, bool W = false>
 struct Prob {
   using Epi = EpiT;
-  static constexpr bool A_MN = AMN, B_MN = BMN, present = true;
+  static constexpr bool A_MN = AMN, B_MN = BMN, present = true, WIDE = W;
   static constexpr int A_HINT = AH, B_HINT = BH;
 };
 
 struct EpiNone;
 struct NoProb {
   using Epi = EpiNone;
-  static constexpr bool A_MN = false, B_MN = false, present = false;
+  static constexpr bool A_MN = false, B_MN = false, present = false, WIDE = false;
   static constexpr int A_HINT = kL2Normal, B_HINT = kL2Normal;
 };
 
@@ -325,6 +339,29 @@ struct RoleState {
   uint32_t acc_phase = 0;
 };
 
+template <class G>
+__device__ __forceinline__ void next_stage(RoleState& st) {
+  if (++st.stage == G::STAGES) { st.stage = 0; st.phase ^= 1u; }
+}
+
+__device__ __forceinline__ void next_acc(RoleState& st) {
+  st.acc ^= 1;
+  if (st.acc == 0) st.acc_phase ^= 1u;
+}
+
+// Column tiles of raster column n: [first, first + count).
+template <class P>
+__device__ __forceinline__ void unit_cols(const ProbArgs& pa, int n, int& first, int& count) {
+  first = n;
+  count = 1;
+  if constexpr (P::WIDE) {
+    if (pa.wide_cols > 0) {
+      first = 2 * n;
+      count = wide_count(n, pa.wide_cols);
+    }
+  }
+}
+
 // TMA producer: all K blocks of every tile of unit u.
 template <class G, bool PAIR, class P>
 __device__ __forceinline__ bool produce_unit(const Smem<G>& L, RoleState& st, uint32_t rank,
@@ -333,17 +370,23 @@ __device__ __forceinline__ bool produce_unit(const Smem<G>& L, RoleState& st, ui
   int m, split, n0, n1;
   decode_unit(pa.raster, u, m, split, n0, n1);
   for (int n = n0; n < n1; ++n) {
+    int c0, nc;
+    unit_cols<P>(pa, n, c0, nc);
     for (int kb = 0; kb < pa.num_kb; ++kb) {
-      if (!mbar_wait_bounded(L.empty(st.stage), st.phase ^ 1u, L.abort_flag)) return false;
-      const uint32_t sa = L.sbase + st.stage * G::STAGE_BYTES;
-      const uint32_t sb = sa + G::A_BYTES;
-      const uint32_t fb = PAIR ? mapa_shared(L.full(st.stage), 0) : L.full(st.stage);
-      if (rank == 0) mbar_arrive_expect_tx(L.full(st.stage), G::TX_BYTES);
-      load_operand<P::A_MN, BM, PAIR>(sa, tA, pa.a_row0 + m * G::TILE_M + (int)rank * BM,
-                                      pa.a_k0 + kb * BK, fb, make_l2_policy(P::A_HINT));
-      load_operand<P::B_MN, G::B_ROWS, PAIR>(sb, tB, pa.b_row0 + n * BN + (int)rank * G::B_ROWS,
-                                             pa.b_k0 + kb * BK, fb, make_l2_policy(P::B_HINT));
-      if (++st.stage == G::STAGES) { st.stage = 0; st.phase ^= 1u; }
+      // stage 1: A and the first column tile's B; stage 2 (wide units): the second B
+      for (int h = 0; h < nc; ++h) {
+        if (!mbar_wait_bounded(L.empty(st.stage), st.phase ^ 1u, L.abort_flag)) return false;
+        const uint32_t sa = L.sbase + st.stage * G::STAGE_BYTES;
+        const uint32_t sb = sa + G::A_BYTES;
+        const uint32_t fb = PAIR ? mapa_shared(L.full(st.stage), 0) : L.full(st.stage);
+        if (rank == 0) mbar_arrive_expect_tx(L.full(st.stage), h == 0 ? G::TX_BYTES : G::TX_B_BYTES);
+        if (h == 0)
+          load_operand<P::A_MN, BM, PAIR>(sa, tA, pa.a_row0 + m * G::TILE_M + (int)rank * BM,
+                                          pa.a_k0 + kb * BK, fb, make_l2_policy(P::A_HINT));
+        load_operand<P::B_MN, G::B_ROWS, PAIR>(sb, tB, pa.b_row0 + (c0 + h) * BN + (int)rank * G::B_ROWS,
+                                               pa.b_k0 + kb * BK, fb, make_l2_policy(P::B_HINT));
+        next_stage<G>(st);
+      }
     }
   }
   return true;
@@ -358,34 +401,52 @@ __device__ __forceinline__ bool mma_unit(const Smem<G>& L, RoleState& st, uint32
   int m, split, n0, n1;
   decode_unit(pa.raster, u, m, split, n0, n1);
   for (int n = n0; n < n1; ++n) {
+    int c0, nc;
+    unit_cols<P>(pa, n, c0, nc);
+    // the unit's accumulators: this one and, for a wide unit, the next
+    RoleState a2 = st;
+    next_acc(a2);
     if (!mbar_wait_bounded(L.tempty(st.acc), st.acc_phase ^ 1u, L.abort_flag)) return false;
+    if (nc == 2 && !mbar_wait_bounded(L.tempty(a2.acc), a2.acc_phase ^ 1u, L.abort_flag)) return false;
     tc_fence_after();
-    const uint32_t d_tmem = tmem_base + st.acc * BN;
+    const uint32_t d0 = tmem_base + st.acc * BN, d1 = tmem_base + a2.acc * BN;
     for (int kb = 0; kb < pa.num_kb; ++kb) {
+      // stage 1 holds A and the first B, stage 2 (wide units) the second B
+      RoleState s2 = st;
+      next_stage<G>(s2);
       if (!mbar_wait_bounded(L.full(st.stage), st.phase, L.abort_flag)) return false;
+      if (nc == 2 && !mbar_wait_bounded(L.full(s2.stage), s2.phase, L.abort_flag)) return false;
       tc_fence_after();
       const uint32_t sa = L.sbase + st.stage * G::STAGE_BYTES;
-      const uint32_t sb = sa + G::A_BYTES;
+      const uint32_t sb0 = sa + G::A_BYTES;
+      const uint32_t sb1 = L.sbase + s2.stage * G::STAGE_BYTES + G::A_BYTES;
 #pragma unroll
       for (int kk = 0; kk < BK / UMMA_K; ++kk) {
         const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-        if constexpr (PAIR)
-          tc_mma_bf16_pair(d_tmem, operand_desc<P::A_MN>(sa, kk), operand_desc<P::B_MN>(sb, kk), idesc, accum);
-        else
-          tc_mma_bf16(d_tmem, operand_desc<P::A_MN>(sa, kk), operand_desc<P::B_MN>(sb, kk), idesc, accum);
+        const uint64_t da = operand_desc<P::A_MN>(sa, kk);
+        if constexpr (PAIR) {
+          tc_mma_bf16_pair(d0, da, operand_desc<P::B_MN>(sb0, kk), idesc, accum);
+          if (nc == 2) tc_mma_bf16_pair(d1, da, operand_desc<P::B_MN>(sb1, kk), idesc, accum);
+        } else {
+          tc_mma_bf16(d0, da, operand_desc<P::B_MN>(sb0, kk), idesc, accum);
+          if (nc == 2) tc_mma_bf16(d1, da, operand_desc<P::B_MN>(sb1, kk), idesc, accum);
+        }
       }
-      if constexpr (PAIR) tc_commit_pair_mc(L.empty(st.stage), 0x3); else tc_commit(L.empty(st.stage));
-      if (++st.stage == G::STAGES) { st.stage = 0; st.phase ^= 1u; }
+      for (int h = 0; h < nc; ++h) {
+        if constexpr (PAIR) tc_commit_pair_mc(L.empty(st.stage), 0x3); else tc_commit(L.empty(st.stage));
+        next_stage<G>(st);
+      }
     }
-    if constexpr (PAIR) tc_commit_pair_mc(L.tfull(st.acc), 0x3); else tc_commit(L.tfull(st.acc));
-    st.acc ^= 1;
-    if (st.acc == 0) st.acc_phase ^= 1u;
+    for (int h = 0; h < nc; ++h) {
+      if constexpr (PAIR) tc_commit_pair_mc(L.tfull(st.acc), 0x3); else tc_commit(L.tfull(st.acc));
+      next_acc(st);
+    }
   }
   return true;
 }
 
 // Epilogue (all 128 threads of warps 2-5): drain each tile of unit u.
-template <class G, bool PAIR, class Epi>
+template <class G, bool PAIR, class P, class Epi>
 __device__ __forceinline__ bool epi_unit(const Smem<G>& L, RoleState& st, uint32_t rank,
                                          uint32_t lane_addr, int row, Epi& epi,
                                          const typename Epi::Params& ep, const CUtensorMap* out,
@@ -396,17 +457,20 @@ __device__ __forceinline__ bool epi_unit(const Smem<G>& L, RoleState& st, uint32
   cx.row_base = m * G::TILE_M + (int)rank * BM;
   epi.begin_unit(ep, grow, split, n0, cx);
   for (int n = n0; n < n1; ++n) {
-    // One outcome for all 128 epilogue threads: tcgen05.ld needs whole
-    // warps and the store path synchronises the four warps.
-    const bool ok = epilogue_bar_and(128, mbar_wait_bounded(L.tfull(st.acc), st.acc_phase, L.abort_flag));
-    if (!ok) return false;
-    tc_fence_after();
-    epi.tile(ep, out, grow, n, lane_addr + st.acc * BN, cx);
-    tc_fence_before();
-    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(L.tempty(st.acc), 0));
-    else mbar_arrive(L.tempty(st.acc));
-    st.acc ^= 1;
-    if (st.acc == 0) st.acc_phase ^= 1u;
+    int c0, nc;
+    unit_cols<P>(pa, n, c0, nc);
+    for (int h = 0; h < nc; ++h) {      // a wide unit's two tiles, one accumulator each
+      // One outcome for all 128 epilogue threads: tcgen05.ld needs whole
+      // warps and the store path synchronises the four warps.
+      const bool ok = epilogue_bar_and(128, mbar_wait_bounded(L.tfull(st.acc), st.acc_phase, L.abort_flag));
+      if (!ok) return false;
+      tc_fence_after();
+      epi.tile(ep, out, grow, c0 + h, lane_addr + st.acc * BN, cx);
+      tc_fence_before();
+      if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(L.tempty(st.acc), 0));
+      else mbar_arrive(L.tempty(st.acc));
+      next_acc(st);
+    }
   }
   epi.end_unit(ep, grow, split);
   return true;
@@ -509,7 +573,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
                                 int u, int) {
       using P = decltype(pt);
       constexpr bool first = std::is_same<P, P0>::value;
-      return epi_unit<G, PAIR>(L, st, rank, lane_addr, row, pick<first>(epi0, epi1), pick<first>(ep0, ep1),
+      return epi_unit<G, PAIR, P>(L, st, rank, lane_addr, row, pick<first>(epi0, epi1), pick<first>(ep0, ep1),
                                first ? &tmO0 : &tmO1, pa, u, cx);
     });
     if (cx.issuer) bulk_wait<0>();          // every TMA store of this CTA has completed

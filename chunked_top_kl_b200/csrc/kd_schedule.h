@@ -60,6 +60,28 @@ KD_HD Raster tile_raster(int64_t m_tiles, int64_t n_tiles, bool bands_fastest) {
   return r;
 }
 
+// Wide units (a problem whose every unit computes two neighbouring 256-column
+// tiles at once): raster column n stands for column tiles [2n, 2n + count)
+// of n_cols, count 2, or 1 for the last of an odd number.
+KD_HD int wide_count(int n, int n_cols) { return 2 * n + 1 < n_cols ? 2 : 1; }
+
+// Whether problem 0 of a joint launch (bands x n_cols tiles of k0 K blocks)
+// should run wide units beside problem 1's U1 units of k1 K blocks on
+// `groups`: a wide unit loads 3/4 of the operand bytes per MMA block, but
+// holds twice the work, so it pays only when the busiest group's share, the
+// larger of its problem-0 units and the launch's average, does not grow, and
+// (measured: slower or no faster otherwise) when every group holds at least
+// one wide unit.
+KD_HD bool wide_pays(int64_t bands, int64_t n_cols, int64_t k0, int64_t U1, int64_t k1, int groups) {
+  const int64_t avg = ceil_div64(bands * n_cols * k0 + U1 * k1, groups);
+  auto busiest = [&](int64_t U0, int64_t c0) {
+    const int64_t own = ceil_div64(U0, groups) * c0;
+    return own > avg ? own : avg;
+  };
+  const int64_t U0w = bands * ceil_div64(n_cols, 2);
+  return n_cols > 1 && U0w >= groups && busiest(U0w, 2 * k0) <= busiest(bands * n_cols, k0);
+}
+
 // Forward pass (and the dZ recompute): a unit is a band and a range of
 // vocabulary tiles whose running log-sum-exp (or teacher-column cursor) one
 // CTA carries.  Picks the number of ranges (<= max_splits; every range is

@@ -238,9 +238,8 @@ cudaError_t launch_one(int slot, int dev, int groups, const CUtensorMap& ta, con
 // Problem 0 round-robin, problem 1 dealt to even out the groups' total K
 // blocks (see joint_plan).
 void plan_second_problem(GemmArgs& a, int groups) {
-  a.joint = joint_plan(a.prob[0].raster.num_units, (int64_t)a.prob[0].raster.tiles_per_split * a.prob[0].num_kb,
-                       a.prob[1].raster.num_units, (int64_t)a.prob[1].raster.tiles_per_split * a.prob[1].num_kb,
-                       groups);
+  a.joint = joint_plan(a.prob[0].raster.num_units, unit_cost(a.prob[0]), a.prob[1].raster.num_units,
+                       unit_cost(a.prob[1]), groups);
 }
 
 // Work groups (CTAs, or CTA pairs) that can be resident at once: one per SM,
@@ -280,7 +279,8 @@ inline int grid_for(const Raster& r, int groups) { return r.num_units < groups ?
 // chunk (keep it); streamed operands use the default priority.
 using ProbFwd = Prob<EpiFwd, false, false, kL2EvictLast, kL2Normal>;  // A = H (K-major), B = W (K-major)
 using ProbDz = Prob<EpiDz, false, false, kL2EvictLast, kL2Normal>;    // A = H chunk, B = W
-using ProbDh = Prob<EpiDh, false, true>;      // A = dZ (K-major over V), B = W (MN-major over d)
+using ProbDh = Prob<EpiDh, false, true, kL2Normal, kL2Normal, true>;   // A = dZ (K-major over V), B = W (MN-major
+                                                                        // over d); wide units (K = V is long)
 using ProbDw = Prob<EpiDw, true, true, kL2Normal, kL2EvictLast>;      // A = dZ^T (MN-major over V), B = H chunk
 using ProbZ32 = Prob<EpiZ32, false, false, kL2EvictLast, kL2Normal>;  // teacher logits, fp32 store: A = Ht, B = Wt
 
@@ -591,15 +591,21 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
       return KD_ERR_CUDA;
 
     // One launch for both gradient products of the chunk:
-    //   problem 0: dH[chunk] = dZ W      (few long tiles, K = V; a band's column
-    //              tiles side by side, so each dZ band is fetched once per wave)
+    //   problem 0: dH[chunk] = dZ W      (few long tiles, K = V; two column tiles
+    //              per unit sharing each dZ load where that keeps the pairs
+    //              balanced; a band's units side by side, so each dZ band is
+    //              fetched once per wave)
     //   problem 1: dW (+)= dZ^T H[chunk] (many short tiles, K = chunk)
     GemmArgs a45{};
     a45.status = status;
     a45.dyn = dyn;
-    a45.prob[0].raster = tile_raster(ceil_div(Cc, GeoP::TILE_M), ceil_div(d, BN), false);
+    const int64_t dh_cols = ceil_div(d, BN), dh_bands = ceil_div(Cc, GeoP::TILE_M);
+    const bool wide = wide_pays(dh_bands, dh_cols, ceil_div(V, BK), ceil_div(V, GeoP::TILE_M) * dh_cols,
+                                ceil_div(Cc, BK), groups);
+    a45.prob[0].raster = tile_raster(dh_bands, wide ? ceil_div(dh_cols, 2) : dh_cols, false);
     a45.prob[0].num_kb = (int)ceil_div(V, BK);
     a45.prob[0].dyn_role = 1;
+    a45.prob[0].wide_cols = wide ? (int)dh_cols : 0;
     a45.prob[1].raster = tile_raster(ceil_div(V, GeoP::TILE_M), ceil_div(d, BN), false);
     a45.prob[1].num_kb = (int)ceil_div(Cc, BK);
     a45.prob[1].b_k0 = hrow0;

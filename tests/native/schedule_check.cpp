@@ -26,6 +26,26 @@ static bool check(const Raster& r, const char* what, long a, long b, long c) {
   return true;
 }
 
+// A wide problem's raster (two column tiles per raster column): every
+// (band, column tile) exactly once.
+static bool check_wide(long m_tiles, long n_cols) {
+  const Raster r = tile_raster(m_tiles, ceil_div64(n_cols, 2), false);
+  std::vector<int> seen((size_t)(m_tiles * n_cols), 0);
+  for (int u = 0; u < r.num_units; ++u) {
+    int m, s, n0, n1;
+    decode_unit(r, u, m, s, n0, n1);
+    for (int n = n0; n < n1; ++n)
+      for (int h = 0; h < wide_count(n, (int)n_cols); ++h) {
+        const long c = 2l * n + h;
+        if (m < 0 || m >= m_tiles || c >= n_cols) { printf("FAIL wide unit %d -> m %d col %ld\n", u, m, c); return false; }
+        seen[(size_t)(m * n_cols + c)]++;
+      }
+  }
+  for (size_t i = 0; i < seen.size(); ++i)
+    if (seen[i] != 1) { printf("FAIL wide tile %zu seen %d (%ld x %ld)\n", i, seen[i], m_tiles, n_cols); return false; }
+  return true;
+}
+
 int main() {
   const long Ns[] = {1, 127, 128, 129, 512, 1000, 4096, 8192, 32768, 65536, 262144};
   const long Vs[] = {1, 24, 255, 256, 257, 4096, 32000, 128256, 201088};
@@ -53,13 +73,14 @@ int main() {
         if (!check(tile_raster(ceil_div64(C, 128), ceil_div64(V, 256), true), "dz", C, V, d)) return 1;
         if (!check(tile_raster(ceil_div64(C, 128), ceil_div64(d, 256), true), "dh", C, V, d)) return 1;
         if (!check(tile_raster(ceil_div64(V, 128), ceil_div64(d, 256), false), "dw", C, V, d)) return 1;
-        cases += 3;
+        if (!check_wide(ceil_div64(C, 256), ceil_div64(d, 256))) return 1;
+        cases += 4;
       }
   // joint launches: every problem-1 unit dealt exactly once; when there are
   // enough of them to even out the groups, no group's K blocks differ from
   // another's by more than 1.5 problem-1 units
-  const long U0s[] = {0, 1, 16, 32, 192, 400};
-  const long k0s[] = {1, 45, 501, 3142};
+  const long U0s[] = {0, 1, 16, 32, 96, 192, 400};
+  const long k0s[] = {1, 45, 501, 3142, 6284};
   const long U1s[] = {0, 1, 12, 9432, 6012};
   const long k1s[] = {1, 16, 64};
   std::vector<int> seen;
@@ -96,7 +117,7 @@ int main() {
   // wave pacing: every counter a group waits on receives exactly the number
   // of arrivals it waits for (else the barrier would time out), all waits
   // on one counter expect the same number, and indices stay in bounds
-  const long ks0[] = {1, 45, 3142};
+  const long ks0[] = {1, 45, 3142, 6284};
   for (long U0 : U0s)
     for (long k0 : ks0)
       for (long U1 : U1s)
@@ -127,6 +148,20 @@ int main() {
               }
             ++cases;
           }
+  // wide dH units on 74 CTA pairs: taken at the 32K GPT-OSS head (4096-token
+  // chunks, d = 2880, V = 201,088: 96 wide units); not at the 8K Llama head's
+  // 2048-token chunks (d = 3072, V = 128,256: 48 wide units) nor at the
+  // long-context sweep's 4096-token chunks (d = 2048: 64 wide units), where
+  // they measured slower or no faster; never with one column tile
+  if (!wide_pays(16, 12, 3142, 786 * 12, 64, 74)) { printf("FAIL wide gptoss\n"); return 1; }
+  if (wide_pays(8, 12, 2004, 501 * 12, 32, 74)) { printf("FAIL wide llama\n"); return 1; }
+  if (wide_pays(16, 8, 2004, 501 * 8, 64, 74)) { printf("FAIL wide sweep\n"); return 1; }
+  if (wide_pays(16, 1, 3142, 786, 64, 74)) { printf("FAIL wide one column\n"); return 1; }
+  // the GPU parity case for wide units with an odd column count (N = 4096,
+  // d = 2640: 11 column tiles, the last 80 columns wide, V = 2048, one
+  // 4096-token chunk) takes them
+  if (!wide_pays(16, 11, 32, 8 * 11, 64, 74)) { printf("FAIL wide odd case\n"); return 1; }
+  cases += 5;
   printf("OK %d\n", cases);
   return 0;
 }

@@ -6,7 +6,11 @@ relative Frobenius 1e-2):
 * a one-column vocabulary (V = K = 1: the teacher and the student agree
   exactly, so the loss and both gradients are zero, the GPU's within
   rounding; lse is the single logit);
-* skipping masked rows with one-token chunks, and with a single kept token.
+* skipping masked rows with one-token chunks, and with a single kept token;
+* the dH product's wide units (two column tiles per unit) with an odd number
+  of column tiles (d = 2640: 11 tiles, the last 80 columns wide and alone in
+  its unit), a shape whose launch takes them (the schedule's CPU check pins
+  that).
 """
 
 from __future__ import annotations
@@ -110,3 +114,7 @@ def test_skip_rows_single_kept_token(kd):
     assert np.all(got["dH"][:299] == 0.0)
     assert math.isclose(got["loss"], ref["term"][299], rel_tol=LOSS_RTOL)
 
+
+def test_wide_dH_units_odd_column_count(kd):
+    x = _inputs(4096, 2640, 2048, 16, seed=12)
+    _parity(_fused(kd, x, 4096), x, "wide dH units, 11 column tiles")
