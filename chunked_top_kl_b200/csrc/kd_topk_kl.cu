@@ -611,8 +611,8 @@ int backward_stage(const void* H, const void* W, const int32_t* topk_idx, const 
     a45.prob[1].b_k0 = hrow0;
     a45.prob[1].dyn_role = 2;
     plan_second_problem(a45, groups);
-    if (a45.prob[1].num_kb >= kPaceKBlocks)     // dW tiles long enough to pace (see wave_slot)
-      a45.wave_sync = jwave + (size_t)(c0 / chunk) * L.jwave_per_chunk;
+    if (a45.prob[1].num_kb >= (wide ? kPaceKBlocksWide : kPaceKBlocks))   // dW tiles long enough to pace
+      a45.wave_sync = jwave + (size_t)(c0 / chunk) * L.jwave_per_chunk;        // (see wave_slot)
     EpiDh::Params e4{};
     e4.row0 = hrow0;
     EpiDw::Params e5{};

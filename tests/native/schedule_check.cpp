@@ -149,19 +149,21 @@ int main() {
             ++cases;
           }
   // wide dH units on 74 CTA pairs: taken at the 32K GPT-OSS head (4096-token
-  // chunks, d = 2880, V = 201,088: 96 wide units); not at the 8K Llama head's
-  // 2048-token chunks (d = 3072, V = 128,256: 48 wide units) nor at the
-  // long-context sweep's 4096-token chunks (d = 2048: 64 wide units), where
-  // they measured slower or no faster; never with one column tile
+  // chunks, d = 2880, V = 201,088: 96 wide units), the 8K Llama head's
+  // 2048-token chunks (d = 3072, V = 128,256: 48) and the long-context sweep's
+  // 4096-token chunks (d = 2048: 64); not at the packed 4K head's 1024-token
+  // chunks (d = 2048, V = 32,000: 16 wide units of twice the launch's average
+  // work), never with one column tile
   if (!wide_pays(16, 12, 3142, 786 * 12, 64, 74)) { printf("FAIL wide gptoss\n"); return 1; }
-  if (wide_pays(8, 12, 2004, 501 * 12, 32, 74)) { printf("FAIL wide llama\n"); return 1; }
-  if (wide_pays(16, 8, 2004, 501 * 8, 64, 74)) { printf("FAIL wide sweep\n"); return 1; }
+  if (!wide_pays(8, 12, 2004, 501 * 12, 32, 74)) { printf("FAIL wide llama\n"); return 1; }
+  if (!wide_pays(16, 8, 2004, 501 * 8, 64, 74)) { printf("FAIL wide sweep\n"); return 1; }
+  if (wide_pays(4, 8, 500, 125 * 8, 16, 74)) { printf("FAIL wide packed\n"); return 1; }
   if (wide_pays(16, 1, 3142, 786, 64, 74)) { printf("FAIL wide one column\n"); return 1; }
   // the GPU parity case for wide units with an odd column count (N = 4096,
   // d = 2640: 11 column tiles, the last 80 columns wide, V = 2048, one
   // 4096-token chunk) takes them
   if (!wide_pays(16, 11, 32, 8 * 11, 64, 74)) { printf("FAIL wide odd case\n"); return 1; }
-  cases += 5;
+  cases += 6;
   printf("OK %d\n", cases);
   return 0;
 }
