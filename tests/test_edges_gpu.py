@@ -10,7 +10,8 @@ relative Frobenius 1e-2):
 * the dH product's wide units (two column tiles per unit) with an odd number
   of column tiles (d = 2640: 11 tiles, the last 80 columns wide and alone in
   its unit), a shape whose launch takes them (the schedule's CPU check pins
-  that).
+  that), all rows and with masked rows skipped (the launch then rebuilds its
+  wide units for the live rows on the device).
 """
 
 from __future__ import annotations
@@ -118,3 +119,14 @@ def test_skip_rows_single_kept_token(kd):
 def test_wide_dH_units_odd_column_count(kd):
     x = _inputs(4096, 2640, 2048, 16, seed=12)
     _parity(_fused(kd, x, 4096), x, "wide dH units, 11 column tiles")
+
+
+def test_wide_dH_units_with_skipped_rows(kd):
+    x = _inputs(4096, 2640, 2048, 16, seed=13, mask="ones")
+    g = torch.Generator().manual_seed(13)
+    x["mask"] = (torch.rand(4096, generator=g) >= 0.3).float()
+    a = _fused(kd, x, 4096, skip=False)
+    b = _fused(kd, x, 4096, skip=True)
+    assert a["loss"] == b["loss"] and np.array_equal(a["lse"], b["lse"]) and np.array_equal(a["dH"], b["dH"])
+    assert _rfro(b["dW"], a["dW"]) <= 1e-5
+    _parity(b, x, "wide dH units, skipped rows")
