@@ -7,8 +7,8 @@
 //                      for each chunk of tokens: [gather_rows ->]
 //                      gemm<EpiDz> -> gemm<EpiDh + EpiDw> [-> scatter_rows]
 //                      (bracketed steps: skipping masked rows)
-// Teacher top-K cache writer: for each chunk, gemm<EpiDw, fp32 store> ->
-//                      topk_select
+// Teacher top-K cache writer: for each chunk, gemm<EpiZ32> (fp32 logits and
+//                      their tile maxima) -> topk_select
 // The fused chunked loss of "Efficient Knowledge Distillation for LLMs"
 // (Japanese summary, method paragraph) projects, normalises and gathers one
 // chunk at a time and recomputes each chunk in the backward pass; here the
