@@ -283,6 +283,7 @@ using ProbDh = Prob<EpiDh, false, true, kL2Normal, kL2Normal, true>;   // A = dZ
                                                                         // over d); wide units (K = V is long)
 using ProbDw = Prob<EpiDw, true, true, kL2Normal, kL2EvictLast>;      // A = dZ^T (MN-major over V), B = H chunk
 using ProbZ32 = Prob<EpiZ32, false, false, kL2EvictLast, kL2Normal>;  // teacher logits, fp32 store: A = Ht, B = Wt
+static_assert(kSelTile == BN, "the select's tile maxima are those of the logits GEMM's column tiles");
 
 // The loss as one call computes it: the teacher logits and their type, T,
 // and the factors of the student-temperature variant (zs on the student

@@ -61,6 +61,8 @@ constexpr int kSelBlock = kSelectThreads * kSelVec;   // float4s per block (8192
 constexpr int kSelSegment = 8;       // blocks between two meetings of the threads
 constexpr int kSelTile = 256;        // columns per tile maximum (the logits GEMM's tile width)
 constexpr int kSelTilesPerBlock = kSelBlock / (kSelTile / 4);   // tiles per block of the tile route
+static_assert(kSelTile / 4 == 64 && kSelectThreads % 64 == 0,
+              "the tile route reads a tile as 64 float4s, one per thread of a 64-thread group");
 constexpr int kSelCap = 2048;        // candidate list (power of two, >= 2 kMaxTopK)
 constexpr int kCandCap = 2048;       // fallback sort buffer (power of two, >= kMaxTopK)
 
@@ -92,10 +94,11 @@ __device__ __forceinline__ void bitonic_sort_desc(unsigned long long* s, int P) 
 }
 
 // Shared state of the selection of one row.  The fallback sorts in the
-// candidate list (its first kCandCap entries) and keeps its own histogram.
+// candidate list (its first kCandCap entries) and keeps its own histogram;
+// until a row falls back, the tile route keeps its selected tiles there.
 struct SelShared {
-  unsigned long long list[kSelCap];     // candidates (key, column)
-  int fhist[4096];                      // the fallback's histogram
+  unsigned long long list[kSelCap];     // candidates (key, column); first, the tile route's tile maxima
+  int fhist[4096];                      // the fallback's histogram, or the tile route's selected tiles
   int hist[2][256];                     // radix histograms of the streaming route (alternating passes)
   int scan[kSelWarps];                  // the fallback's per-warp tie counts
   uint32_t wkey[kSelWarps];
@@ -103,6 +106,7 @@ struct SelShared {
   uint32_t prefix, mask;
 };
 static_assert(kCandCap <= kSelCap, "the fallback sorts in the candidate list");
+static_assert(kSelCap <= 4096, "the tile route (at most kSelCap tiles) lists its tiles in fhist");
 
 __device__ __forceinline__ unsigned long long* fallback_sort(SelShared& S) { return S.list; }
 __device__ __forceinline__ int* fallback_hist(SelShared& S) { return S.fhist; }
